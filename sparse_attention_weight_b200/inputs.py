@@ -1,0 +1,206 @@
+"""Seeded synthetic inputs for the DSA path.
+
+This module only draws random numbers and stores them in the input formats
+(FP8 E4M3 bytes, bf16 bit patterns, fp32).  It holds none of the method's
+arithmetic, so both the CUDA path and the CPU oracle can take their inputs
+from it.
+
+Streams.  Every tensor is drawn in row chunks of ``ROW_CHUNK`` rows; chunk c
+of tensor ``tid`` in sequence ``b`` comes from
+``numpy.random.default_rng([seed, cfg_id, tid, b, c])``, so any row can be
+regenerated on its own (the oracle samples rows of the large workloads).
+Tensor ids: 0 indexer query q_I, 1 indexer key k_I, 2 indexer head weights w,
+3 MLA query Q, 4 latent KV rows, 5 decode context lengths.
+
+Rows of per-query tensors are numbered by position for prefill (queries are
+positions 0..L-1 of sequence 0) and by the query's ordinal inside its
+sequence for decode.  Cache rows are numbered by position.
+
+Quantisation: N(0,1) float32 values are clamped to +-448 and cast to E4M3 by
+PyTorch's round-to-nearest-even cast; bf16 tensors use PyTorch's RNE cast.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from .configs import D_INDEX, D_QK, Workload
+
+ROW_CHUNK = 256
+E4M3_MAX = 448.0
+
+T_QIDX, T_KIDX, T_W, T_Q, T_KV, T_LEN = 0, 1, 2, 3, 4, 5
+
+
+def _chunk_rows(seed: int, cfg_id: int, tid: int, seq: int, row0: int, nrows: int,
+                row_shape: tuple[int, ...], std: float = 1.0) -> np.ndarray:
+    """float32 N(0, std^2) rows [row0, row0+nrows) of one tensor of one sequence."""
+    out = np.empty((nrows,) + tuple(row_shape), dtype=np.float32)
+    if nrows == 0:
+        return out
+    c0, c1 = row0 // ROW_CHUNK, (row0 + nrows - 1) // ROW_CHUNK
+    for c in range(c0, c1 + 1):
+        rng = np.random.default_rng([seed, cfg_id, tid, seq, c])
+        chunk = rng.standard_normal((ROW_CHUNK,) + tuple(row_shape), dtype=np.float32)
+        if std != 1.0:
+            chunk *= np.float32(std)
+        lo = max(row0, c * ROW_CHUNK)
+        hi = min(row0 + nrows, (c + 1) * ROW_CHUNK)
+        out[lo - row0:hi - row0] = chunk[lo - c * ROW_CHUNK:hi - c * ROW_CHUNK]
+    return out
+
+
+def to_e4m3_bytes(x: np.ndarray) -> np.ndarray:
+    """float32 -> E4M3 bytes (uint8) via PyTorch's RNE cast, clamped to +-448."""
+    t = torch.from_numpy(np.clip(np.ascontiguousarray(x, dtype=np.float32), -E4M3_MAX, E4M3_MAX))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns (uint16) via PyTorch's RNE cast."""
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+@dataclass
+class Batch:
+    """Host copy of the batch description (mirrors ``dsa_batch`` in dsa.h)."""
+    kv_offset: np.ndarray   # int64 [B]   first cache row of sequence b
+    kv_len: np.ndarray      # int32 [B]   cache rows of sequence b
+    q_seq: np.ndarray       # int32 [T]   sequence of query t
+    q_pos: np.ndarray       # int32 [T]   position of query t; keys 0..q_pos visible
+    q_row: np.ndarray       # int32 [T]   row of query t in its sequence's query streams
+
+    @property
+    def num_seqs(self) -> int:
+        return int(self.kv_len.shape[0])
+
+    @property
+    def num_q(self) -> int:
+        return int(self.q_pos.shape[0])
+
+    @property
+    def max_kv_len(self) -> int:
+        return int(self.kv_len.max()) if self.kv_len.size else 0
+
+    @property
+    def max_q_per_seq(self) -> int:
+        if self.q_seq.size == 0:
+            return 0
+        return int(np.bincount(self.q_seq, minlength=self.num_seqs).max())
+
+    @property
+    def total_rows(self) -> int:
+        return int(self.kv_len.sum())
+
+
+def decode_lengths(wl: Workload, seed: int = 0) -> np.ndarray:
+    """Context lengths of a decode workload (uniform integers, inclusive bounds)."""
+    rng = np.random.default_rng([seed, wl.cfg_id, T_LEN])
+    return rng.integers(wl.ctx_min, wl.ctx_max, size=wl.batch, endpoint=True).astype(np.int32)
+
+
+def make_batch(wl: Workload, seed: int = 0, chunk_index: int | None = None) -> Batch:
+    """Batch description of one call of the workload.
+
+    Prefill: one sequence of ``seq_len`` rows, queries at positions 0..L-1.
+    Chunked prefill: call ``chunk_index`` c holds queries [c*chunk, (c+1)*chunk)
+    against the cache prefix [0, (c+1)*chunk).
+    Decode: ``batch`` sequences; the context length n includes the new
+    token(s), so the q_per_seq queries sit at positions n-q_per_seq .. n-1.
+    """
+    if wl.kind == "prefill":
+        L = wl.seq_len
+        return Batch(np.zeros(1, np.int64), np.array([L], np.int32), np.zeros(L, np.int32),
+                     np.arange(L, dtype=np.int32), np.arange(L, dtype=np.int32))
+    if wl.kind == "chunked_prefill":
+        c = 0 if chunk_index is None else int(chunk_index)
+        lo, hi = c * wl.chunk, (c + 1) * wl.chunk
+        if hi > wl.seq_len or c < 0:
+            raise ValueError("chunk index out of range")
+        pos = np.arange(lo, hi, dtype=np.int32)
+        return Batch(np.zeros(1, np.int64), np.array([hi], np.int32), np.zeros(hi - lo, np.int32),
+                     pos, pos.copy())
+    if wl.kind == "decode":
+        lens = decode_lengths(wl, seed)
+        off = np.zeros(wl.batch, np.int64)
+        off[1:] = np.cumsum(lens[:-1].astype(np.int64))
+        qs = np.repeat(np.arange(wl.batch, dtype=np.int32), wl.q_per_seq)
+        j = np.tile(np.arange(wl.q_per_seq, dtype=np.int32), wl.batch)
+        pos = (lens[qs] - wl.q_per_seq + j).astype(np.int32)
+        return Batch(off, lens, qs, pos, j)
+    raise ValueError(f"unknown workload kind {wl.kind}")
+
+
+def query_rows(wl: Workload, batch: Batch, which: str, seed: int = 0,
+               queries: np.ndarray | None = None) -> np.ndarray:
+    """Per-query tensor for the given query indices (all queries by default).
+
+    which: "q_idx" -> uint8 [n, H_I, 128]; "w" -> float32 [n, H_I];
+    "q" -> uint16 bf16 bits [n, H, 576].
+    """
+    if queries is None:
+        queries = np.arange(batch.num_q)
+    queries = np.asarray(queries, dtype=np.int64)
+    if which == "q_idx":
+        tid, shape, std = T_QIDX, (wl.h_index, D_INDEX), 1.0
+    elif which == "w":
+        tid, shape, std = T_W, (wl.h_index,), 1.0 / np.sqrt(wl.h_index)
+    elif which == "q":
+        tid, shape, std = T_Q, (wl.heads, D_QK), 1.0
+    else:
+        raise ValueError(which)
+    out = np.empty((queries.size,) + shape, np.float32)
+    # group consecutive queries of one sequence with consecutive rows
+    i = 0
+    while i < queries.size:
+        t = queries[i]
+        b, r = int(batch.q_seq[t]), int(batch.q_row[t])
+        j = i + 1
+        while (j < queries.size and batch.q_seq[queries[j]] == b
+               and batch.q_row[queries[j]] == r + (j - i)):
+            j += 1
+        out[i:j] = _chunk_rows(seed, wl.cfg_id, tid, b, r, j - i, shape, std)
+        i = j
+    if which == "q_idx":
+        return to_e4m3_bytes(out)
+    if which == "q":
+        return to_bf16_bits(out)
+    return out
+
+
+def cache_rows(wl: Workload, batch: Batch, which: str, seed: int = 0,
+               seq: int | None = None, row0: int = 0, nrows: int | None = None) -> np.ndarray:
+    """Cache tensor rows.  With ``seq`` given: rows [row0, row0+nrows) of that
+    sequence.  Otherwise: the whole packed cache of the batch (sequence b at
+    rows kv_offset[b] ..).
+
+    which: "k_idx" -> uint8 [rows, 128]; "kv" -> uint16 bf16 bits [rows, 576].
+    """
+    if which == "k_idx":
+        tid, shape, cast = T_KIDX, (D_INDEX,), to_e4m3_bytes
+    elif which == "kv":
+        tid, shape, cast = T_KV, (D_QK,), to_bf16_bits
+    else:
+        raise ValueError(which)
+    if seq is not None:
+        n = int(batch.kv_len[seq]) - row0 if nrows is None else nrows
+        return cast(_chunk_rows(seed, wl.cfg_id, tid, seq, row0, n, shape))
+    parts = [cast(_chunk_rows(seed, wl.cfg_id, tid, b, 0, int(batch.kv_len[b]), shape))
+             for b in range(batch.num_seqs)]
+    return np.concatenate(parts, axis=0) if parts else np.empty((0,) + shape, np.uint8)
+
+
+def make_inputs(wl: Workload, seed: int = 0, chunk_index: int | None = None) -> dict:
+    """Every input of one call of the workload, as host numpy arrays."""
+    batch = make_batch(wl, seed, chunk_index)
+    return {
+        "batch": batch,
+        "q_idx": query_rows(wl, batch, "q_idx", seed),
+        "w": query_rows(wl, batch, "w", seed),
+        "q": query_rows(wl, batch, "q", seed),
+        "k_idx": cache_rows(wl, batch, "k_idx", seed),
+        "kv": cache_rows(wl, batch, "kv", seed),
+    }
