@@ -1,0 +1,170 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention hot path.
+ *
+ * The method (pages "一文讀懂DeepSeek-V3.2核心技術DSA", section "DSA 的四步工作流程";
+ * "DeepSeek-V3.2加速技术详解", sections 3.1-3.2; "DeepSeek 稀疏注意力路线", section
+ * "DeepSeek-V3.2：DSA / 两阶段流程") runs three steps per query token t:
+ *   1. lightning indexer:  I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j,:] . k_I[s,:])
+ *      over the visible keys s <= pos_t, FP8 E4M3 queries/keys of 128 dims;
+ *   2. fine-grained top-k: the k keys with the highest I (all of them when the
+ *      context holds <= k keys);
+ *   3. sparse MLA in MQA form: softmax attention of every query head over only
+ *      the selected rows of the shared latent cache (576-dim key = 512 latent +
+ *      64 RoPE; the value is the 512-dim latent).
+ *
+ * Conventions for every call
+ *   - Pointers marked (device) are CUDA device pointers; everything else is host.
+ *   - The caller owns every buffer and the stream.  The library allocates
+ *     nothing and keeps no per-call state; it creates TMA descriptors on the host
+ *     per call.  All calls are asynchronous on `stream` (a cudaStream_t passed as
+ *     void*; NULL = the legacy default stream) and never synchronise, except
+ *     dsa_read_device_status.
+ *   - Arguments are checked on the host before any launch; on a failed check
+ *     nothing is launched or written and the status says why.
+ *   - Errors the host cannot see (a query position beyond its sequence, an index
+ *     out of range, a bounded wait that ran out) are recorded as bit flags in a
+ *     status word at the start of the workspace `ws`; each call clears the word
+ *     when it starts.  Read it with dsa_read_device_status.
+ *   - Batches: sequence b owns the cache rows kv_offset[b] .. kv_offset[b] +
+ *     kv_len[b] - 1 of k_idx and kv (rows of one sequence are contiguous).
+ *     Query t belongs to sequence q_seq[t] and sees its keys 0 .. q_pos[t]
+ *     (n_t = q_pos[t] + 1 keys; causal and inclusive).  Key and selection
+ *     indices are local to the sequence.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_ABI_VERSION 1
+
+/* Fixed widths of the method (one indexer key per token of 128 dims; latent 512
+ * + RoPE 64; value = latent). */
+#define DSA_D_INDEX 128
+#define DSA_D_QK 576
+#define DSA_D_V 512
+
+typedef enum dsa_status {
+  DSA_OK = 0,
+  DSA_ERR_INVALID_ARGUMENT = 1,   /* null pointer, negative size, inconsistent sizes */
+  DSA_ERR_UNSUPPORTED = 2,        /* a size outside the supported shapes below */
+  DSA_ERR_WORKSPACE_TOO_SMALL = 3,/* ws_bytes < dsa_workspace_size(...) */
+  DSA_ERR_CUDA = 4,               /* a CUDA runtime/driver call or launch failed */
+  DSA_ERR_DEVICE = 5              /* dsa_read_device_status found a device flag */
+} dsa_status;
+
+/* Bit flags of the device status word. */
+#define DSA_DEV_BAD_QUERY 1u      /* q_seq out of [0,B) or q_pos out of [0, kv_len) */
+#define DSA_DEV_BAD_INDEX 2u      /* a selected index >= kv_len of its sequence */
+#define DSA_DEV_TIMEOUT 4u        /* a bounded in-kernel wait expired; results invalid */
+
+typedef struct dsa_batch {
+  int32_t num_seqs;        /* B >= 1 */
+  int32_t num_q;           /* T >= 0 query tokens in this call */
+  int32_t max_kv_len;      /* >= every kv_len[b]; sizes grids and score rows */
+  int32_t max_q_per_seq;   /* >= the number of queries of any one sequence (a grouping hint
+                              for the indexer); 0 means "unknown" (taken as num_q) */
+  int64_t kv_rows;         /* rows held by the k_idx / kv buffers (>= kv_offset[b] + kv_len[b]) */
+  const int64_t *kv_offset;/* (device) [B] first cache row of sequence b */
+  const int32_t *kv_len;   /* (device) [B] cache rows of sequence b */
+  const int32_t *q_seq;    /* (device) [T] sequence of query t */
+  const int32_t *q_pos;    /* (device) [T] position of query t, 0 <= q_pos < kv_len */
+} dsa_batch;
+
+/* Operation codes for dsa_workspace_size. */
+#define DSA_OP_INDEXER 0
+#define DSA_OP_TOPK 1
+#define DSA_OP_SPARSE_MLA 2
+#define DSA_OP_FORWARD 3
+
+/*
+ * Bytes of workspace `ws` an operation needs (always >= 256: the status word and
+ * a small plan live at its start).  `ld` is the score row stride (elements) for
+ * DSA_OP_FORWARD (0 = the default, max_kv_len rounded up to a multiple of 4).
+ * Returns 0 for an invalid op or batch.
+ */
+size_t dsa_workspace_size(int op, const dsa_batch *batch, int H_I, int H, int k, int64_t ld);
+
+/*
+ * Step 1, lightning indexer ("四步工作流程" 第二步 索引器評分; "两阶段流程" 1).
+ *   q_idx  (device) E4M3 bytes [T, H_I, 128], row-major
+ *   k_idx  (device) E4M3 bytes [total cache rows, 128]
+ *   w      (device) fp32 [T, H_I] per-head weights (any scale is folded into w)
+ *   scores (device) fp32 [T, ld]: scores[t*ld + s] = I[t,s] for s < n_t.
+ *          Entries s >= n_t are not written.
+ * Supported: H_I in {4, 8, 16, 32, 64}; ld >= max_kv_len, ld % 4 == 0;
+ * the address of every buffer 16-byte aligned.  FP8 products are accumulated
+ * in fp32 by the tensor cores; the ReLU, per-head weighting and head sum run
+ * in fp32.
+ */
+dsa_status dsa_indexer_scores(const dsa_batch *batch, const uint8_t *q_idx, const uint8_t *k_idx,
+                              const float *w, int H_I, float *scores, int64_t ld,
+                              void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Step 2, top-k selection ("四步工作流程" 第三步 Top-k 選擇; "两阶段流程" 2).
+ *   scores (device) fp32 [T, ld] as written by dsa_indexer_scores (only s < n_t read)
+ *   idx    (device) int32 [T, k]: if n_t <= k, 0..n_t-1; otherwise the k keys with
+ *          the largest score, equal scores going to the lower index (-0.0 == +0.0).
+ *          Ascending index order, padded with -1 to width k.  Exact (radix select
+ *          on the fp32 bit patterns); NaN scores are not supported.
+ * Supported: 1 <= k <= 2048; ld >= max_kv_len, ld % 4 == 0; scores 16-byte aligned.
+ */
+dsa_status dsa_topk(const dsa_batch *batch, const float *scores, int64_t ld, int k, int32_t *idx,
+                    void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Step 3, sparse MLA in MQA form ("四步工作流程" 第四步 執行稀疏 MLA; "DeepSeek-V3.2
+ * 加速技术详解" 3.1 MQA版MLA and 3.2 hard selection).
+ *   q   (device) bf16 bits [T, H, 576] query heads (latent part then RoPE part)
+ *   kv  (device) bf16 bits [total cache rows, 576]; the value of a row is its
+ *       first 512 entries
+ *   idx (device) int32 [T, k] local row indices; -1 entries are skipped
+ *   out (device) bf16 bits [T, H, 512] = sum_i p_i * kv[row_i, :512] with
+ *       p = softmax_i(sm_scale * q . kv[row_i, :576]) in fp32
+ *   lse (device, may be NULL) fp32 [T, H] natural-log log-sum-exp of the scaled
+ *       logits; a query with no valid index gets out = 0 and lse = -inf.
+ * Supported: H in {8, 16, ..., 128} (multiples of 8, padded to 128 inside);
+ * 1 <= k <= 2048.
+ */
+dsa_status dsa_sparse_mla(const dsa_batch *batch, const uint16_t *q, const uint16_t *kv,
+                          const int32_t *idx, int k, int H, float sm_scale, uint16_t *out,
+                          float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Steps 1-3 on one stream ("四步工作流程" 第二步 to 第四步).  Scores and selected
+ * indices live in `ws` (row stride: max_kv_len rounded up to 4).
+ * Arguments as in the three calls above.
+ */
+dsa_status dsa_forward(const dsa_batch *batch, const uint8_t *q_idx, const uint8_t *k_idx,
+                       const float *w, int H_I, const uint16_t *q, const uint16_t *kv, int H, int k,
+                       float sm_scale, uint16_t *out, float *lse, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* Pointers into a forward workspace (for inspection by tests): scores [T, ld]
+ * fp32 and idx [T, k] int32.  Returns DSA_ERR_INVALID_ARGUMENT on bad input. */
+dsa_status dsa_forward_ws_views(const dsa_batch *batch, int H_I, int H, int k, void *ws,
+                                float **scores, int64_t *ld, int32_t **idx);
+
+/*
+ * Synchronises `stream`, copies the device status word of `ws` into *flags and
+ * returns DSA_OK if it is zero, DSA_ERR_DEVICE otherwise.
+ */
+dsa_status dsa_read_device_status(const void *ws, uint32_t *flags, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *dsa_status_string(dsa_status status);
+
+/* DSA_ABI_VERSION of the built library. */
+int dsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

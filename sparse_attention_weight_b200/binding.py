@@ -1,0 +1,192 @@
+"""Thin ctypes binding of libdsa.so (include/dsa.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch tensors on the CUDA device; their data pointers
+and the current torch stream are passed to the C ABI.  A missing library is an
+error (there is no fallback).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa.so")
+
+DSA_OK = 0
+STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARGUMENT", 2: "DSA_ERR_UNSUPPORTED",
+                3: "DSA_ERR_WORKSPACE_TOO_SMALL", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_DEVICE"}
+DEV_BAD_QUERY, DEV_BAD_INDEX, DEV_TIMEOUT = 1, 2, 4
+OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD = 0, 1, 2, 3
+
+EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward",
+           "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version")
+
+
+class DsaError(RuntimeError):
+    def __init__(self, fn: str, status: int, flags: int | None = None):
+        self.status = status
+        self.flags = flags
+        msg = f"{fn} returned {STATUS_NAMES.get(status, status)}"
+        if flags is not None:
+            msg += f" (device flags 0x{flags:x})"
+        super().__init__(msg)
+
+
+class DsaBatch(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("num_q", ctypes.c_int32), ("max_kv_len", ctypes.c_int32),
+                ("max_q_per_seq", ctypes.c_int32), ("kv_rows", ctypes.c_int64),
+                ("kv_offset", ctypes.c_void_p), ("kv_len", ctypes.c_void_p), ("q_seq", ctypes.c_void_p),
+                ("q_pos", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libdsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m sparse_attention_weight_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz, i32, i64, f32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+        bp = ctypes.POINTER(DsaBatch)
+        L.dsa_workspace_size.argtypes = [i32, bp, i32, i32, i32, i64]
+        L.dsa_workspace_size.restype = sz
+        L.dsa_indexer_scores.argtypes = [bp, vp, vp, vp, i32, vp, i64, vp, sz, vp]
+        L.dsa_topk.argtypes = [bp, vp, i64, i32, vp, vp, sz, vp]
+        L.dsa_sparse_mla.argtypes = [bp, vp, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
+        L.dsa_forward.argtypes = [bp, vp, vp, vp, i32, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
+        L.dsa_forward_ws_views.argtypes = [bp, i32, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(i64),
+                                           ctypes.POINTER(vp)]
+        L.dsa_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
+        L.dsa_status_string.argtypes = [i32]
+        L.dsa_status_string.restype = ctypes.c_char_p
+        L.dsa_abi_version.restype = i32
+        for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward", "dsa_forward_ws_views",
+                   "dsa_read_device_status"):
+            getattr(L, fn).restype = i32
+        _lib = L
+    return _lib
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the DSA library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+@dataclass
+class DeviceBatch:
+    """Device arrays of a batch description plus the ctypes struct pointing at them."""
+    kv_offset: torch.Tensor
+    kv_len: torch.Tensor
+    q_seq: torch.Tensor
+    q_pos: torch.Tensor
+    struct: DsaBatch
+
+    @classmethod
+    def from_host(cls, b, device, kv_rows: int | None = None, max_kv_len: int | None = None,
+                  max_q_per_seq: int | None = None) -> "DeviceBatch":
+        """`b` has numpy kv_offset, kv_len, q_seq, q_pos (e.g. inputs.Batch)."""
+        off = torch.as_tensor(np.asarray(b.kv_offset, np.int64), device=device)
+        ln = torch.as_tensor(np.asarray(b.kv_len, np.int32), device=device)
+        qs = torch.as_tensor(np.asarray(b.q_seq, np.int32), device=device)
+        qp = torch.as_tensor(np.asarray(b.q_pos, np.int32), device=device)
+        kv_len = np.asarray(b.kv_len)
+        if kv_rows is None:
+            kv_rows = int((np.asarray(b.kv_offset) + kv_len).max()) if kv_len.size else 0
+        if max_kv_len is None:
+            max_kv_len = int(kv_len.max()) if kv_len.size else 1
+        if max_q_per_seq is None:
+            qsn = np.asarray(b.q_seq)
+            max_q_per_seq = int(np.bincount(qsn).max()) if qsn.size else 0
+        st = DsaBatch(len(kv_len), len(np.asarray(b.q_pos)), max_kv_len, max_q_per_seq, kv_rows,
+                      off.data_ptr(), ln.data_ptr(), qs.data_ptr(), qp.data_ptr())
+        return cls(off, ln, qs, qp, st)
+
+
+def workspace_size(op: int, batch: DeviceBatch, H_I: int = 64, H: int = 128, k: int = 2048, ld: int = 0) -> int:
+    n = lib().dsa_workspace_size(op, ctypes.byref(batch.struct), H_I, H, k, ld)
+    if n == 0:
+        raise DsaError("dsa_workspace_size", 1)
+    return int(n)
+
+
+def workspace(op: int, batch: DeviceBatch, H_I: int = 64, H: int = 128, k: int = 2048, ld: int = 0,
+              device="cuda") -> torch.Tensor:
+    return torch.empty(workspace_size(op, batch, H_I, H, k, ld), dtype=torch.uint8, device=device)
+
+
+def _check(fn: str, status: int):
+    if status != DSA_OK:
+        raise DsaError(fn, status)
+
+
+def dsa_indexer_scores(batch: DeviceBatch, q_idx, k_idx, w, H_I: int, scores, ld: int, ws, stream=None):
+    _check("dsa_indexer_scores", lib().dsa_indexer_scores(
+        ctypes.byref(batch.struct), _ptr(q_idx), _ptr(k_idx), _ptr(w), H_I, _ptr(scores), ld, _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def dsa_topk(batch: DeviceBatch, scores, ld: int, k: int, idx, ws, stream=None):
+    _check("dsa_topk", lib().dsa_topk(ctypes.byref(batch.struct), _ptr(scores), ld, k, _ptr(idx), _ptr(ws),
+                                      ws.numel(), _stream(stream)))
+
+
+def dsa_sparse_mla(batch: DeviceBatch, q, kv, idx, k: int, H: int, sm_scale: float, out, lse, ws, stream=None):
+    _check("dsa_sparse_mla", lib().dsa_sparse_mla(
+        ctypes.byref(batch.struct), _ptr(q), _ptr(kv), _ptr(idx), k, H, sm_scale, _ptr(out), _ptr(lse), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def dsa_forward(batch: DeviceBatch, q_idx, k_idx, w, H_I: int, q, kv, H: int, k: int, sm_scale: float, out, lse,
+                ws, stream=None):
+    _check("dsa_forward", lib().dsa_forward(
+        ctypes.byref(batch.struct), _ptr(q_idx), _ptr(k_idx), _ptr(w), H_I, _ptr(q), _ptr(kv), H, k, sm_scale,
+        _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def forward_ws_views(batch: DeviceBatch, H_I: int, H: int, k: int, ws) -> tuple[int, int, int]:
+    """(scores pointer, ld, idx pointer) inside a forward workspace."""
+    s, i = ctypes.c_void_p(), ctypes.c_void_p()
+    ld = ctypes.c_int64()
+    _check("dsa_forward_ws_views", lib().dsa_forward_ws_views(ctypes.byref(batch.struct), H_I, H, k, _ptr(ws),
+                                                              ctypes.byref(s), ctypes.byref(ld), ctypes.byref(i)))
+    return s.value, ld.value, i.value
+
+
+def read_device_status(ws, stream=None) -> int:
+    """Synchronises the stream and returns the device status flags of `ws`."""
+    flags = ctypes.c_uint32(0)
+    st = lib().dsa_read_device_status(_ptr(ws), ctypes.byref(flags), _stream(stream))
+    if st not in (DSA_OK, 5):
+        raise DsaError("dsa_read_device_status", st)
+    return int(flags.value)
+
+
+def bits_to_tensor(a: np.ndarray, device) -> torch.Tensor:
+    """Host numpy array (uint8 / uint16 bit patterns / float32 / int) -> device tensor of the same bits."""
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def tensor_to_bits(t: torch.Tensor) -> np.ndarray:
+    a = t.cpu().numpy()
+    if t.dtype == torch.int16:
+        return a.view(np.uint16)
+    return a

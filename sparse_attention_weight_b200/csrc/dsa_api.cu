@@ -1,0 +1,333 @@
+// C ABI of the DSA hot path (declared in include/dsa.h): argument checks,
+// workspace layout, TMA descriptors and launches on the caller's stream.
+#include <cstring>
+#include <mutex>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes, 128-byte swizzled boxes.
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, size_t elem, const void* base, uint64_t cols,
+                 uint64_t rows, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * elem};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool batch_ok(const dsa_batch* b) {
+  if (!b) return false;
+  if (b->num_seqs < 1 || b->num_q < 0 || b->max_kv_len < 1 || b->max_q_per_seq < 0 || b->kv_rows < 0) return false;
+  if (b->num_q > 0 && (!b->kv_offset || !b->kv_len || !b->q_seq || !b->q_pos)) return false;
+  return true;
+}
+
+bool hi_ok(int H_I) { return H_I == 4 || H_I == 8 || H_I == 16 || H_I == 32 || H_I == 64; }
+bool h_ok(int H) { return H >= 8 && H <= 128 && H % 8 == 0; }
+bool k_ok(int k) { return k >= 1 && k <= 2048; }
+
+int64_t default_ld(const dsa_batch* b) { return (static_cast<int64_t>(b->max_kv_len) + 3) / 4 * 4; }
+
+// Query tokens per indexer group: a power of two covering the queries of one
+// sequence, with the MMA N = G * H_I in [16, 256].
+int indexer_group(const dsa_batch* b, int H_I) {
+  int want = b->max_q_per_seq > 0 ? b->max_q_per_seq : b->num_q;
+  int g = 1;
+  while (g < want && g * H_I < 256) g <<= 1;
+  while (g * H_I < 16) g <<= 1;
+  return g;
+}
+
+// Splits of each query's index list in the sparse-MLA kernel: enough CTA pairs
+// to fill one wave of the SMs when there are few queries.
+int mla_splits(const dsa_batch* b, int k) {
+  const int pairs = num_sms() / 2;
+  const int blocks = (k + 127) / 128;
+  if (b->num_q <= 0) return 1;
+  int s = pairs / b->num_q;
+  if (s < 1) s = 1;
+  if (s > blocks) s = blocks;
+  if (s > 16) s = 16;
+  return s;
+}
+
+size_t plan_bytes(const dsa_batch* b) { return align_up((6 * static_cast<size_t>(b->num_q) + 2) * sizeof(int32_t)); }
+
+struct WsLayout {
+  uint32_t* status;
+  int32_t* plan;
+  float* part_o;
+  float* part_lse;
+  float* scores;
+  int32_t* idx;
+  size_t bytes;
+};
+
+WsLayout layout(void* ws, int op, const dsa_batch* b, int H, int k, int64_t ld) {
+  WsLayout L{};
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  size_t off = kWsHeader;
+  L.status = reinterpret_cast<uint32_t*>(p);
+  if (op == DSA_OP_INDEXER || op == DSA_OP_FORWARD) {
+    L.plan = reinterpret_cast<int32_t*>(p + off);
+    off += plan_bytes(b);
+  }
+  if (op == DSA_OP_SPARSE_MLA || op == DSA_OP_FORWARD) {
+    const int s = mla_splits(b, k);
+    if (s > 1) {
+      const size_t rows = static_cast<size_t>(b->num_q) * s * H;
+      L.part_o = reinterpret_cast<float*>(p + off);
+      off += align_up(rows * DSA_D_V * sizeof(float));
+      L.part_lse = reinterpret_cast<float*>(p + off);
+      off += align_up(rows * sizeof(float));
+    }
+  }
+  if (op == DSA_OP_FORWARD) {
+    L.scores = reinterpret_cast<float*>(p + off);
+    off += align_up(static_cast<size_t>(b->num_q) * ld * sizeof(float));
+    L.idx = reinterpret_cast<int32_t*>(p + off);
+    off += align_up(static_cast<size_t>(b->num_q) * k * sizeof(int32_t));
+  }
+  L.bytes = off;
+  return L;
+}
+
+dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
+
+dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* k_idx, const float* w, int H_I,
+                       float* scores, int64_t ld, const WsLayout& L, cudaStream_t st) {
+  if (b->num_q == 0) return DSA_OK;
+  const int G = indexer_group(b, H_I);
+  CUtensorMap tq, tk;
+  if (!make_map_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q_idx, DSA_D_INDEX,
+                   static_cast<uint64_t>(b->num_q) * H_I, DSA_D_INDEX, static_cast<uint32_t>(G * H_I)))
+    return DSA_ERR_CUDA;
+  if (!make_map_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k_idx, DSA_D_INDEX,
+                   static_cast<uint64_t>(b->kv_rows > 0 ? b->kv_rows : 1), DSA_D_INDEX, 128))
+    return DSA_ERR_CUDA;
+  const int T = b->num_q;
+  IndexerParams p{};
+  p.w = w;
+  p.scores = scores;
+  p.ld = ld;
+  p.q_seq = b->q_seq;
+  p.q_pos = b->q_pos;
+  p.kv_offset = b->kv_offset;
+  p.kv_len = b->kv_len;
+  int32_t* plan = L.plan;
+  p.group_q0 = plan;
+  p.group_cnt = plan + T;
+  p.group_seq = plan + 2 * T;
+  p.group_tiles = plan + 3 * T;
+  p.item_off = plan + 4 * T;           // T + 1 entries
+  p.ngroups = plan + 5 * T + 1;
+  p.q_nvis = plan + 5 * T + 2;         // T entries (plan has 6T + 2)
+  p.status = L.status;
+  p.G = G;
+  p.max_kv_len = b->max_kv_len;
+  return cuda_status(launch_indexer(tq, tk, p, H_I, T, b->num_seqs, b->kv_rows, num_sms(), st));
+}
+
+dsa_status run_topk(const dsa_batch* b, const float* scores, int64_t ld, int k, int32_t* idx, const WsLayout& L,
+                    cudaStream_t st) {
+  TopkParams p{};
+  p.scores = scores;
+  p.ld = ld;
+  p.idx = idx;
+  p.k = k;
+  p.q_seq = b->q_seq;
+  p.q_pos = b->q_pos;
+  p.kv_len = b->kv_len;
+  p.num_seqs = b->num_seqs;
+  p.max_kv_len = b->max_kv_len;
+  p.status = L.status;
+  return cuda_status(launch_topk(p, b->num_q, st));
+}
+
+dsa_status run_mla(const dsa_batch* b, const uint16_t* q, const uint16_t* kv, const int32_t* idx, int k, int H,
+                   float sm_scale, uint16_t* out, float* lse, const WsLayout& L, cudaStream_t st) {
+  if (b->num_q == 0) return DSA_OK;
+  CUtensorMap tq;
+  if (!make_map_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q, DSA_D_QK, static_cast<uint64_t>(b->num_q) * H, 64,
+                   64))
+    return DSA_ERR_CUDA;
+  MlaParams p{};
+  p.q = q;
+  p.kv = kv;
+  p.idx = idx;
+  p.k = k;
+  p.H = H;
+  p.sm_scale = sm_scale;
+  p.sm_scale_log2 = sm_scale * 1.4426950408889634f;
+  p.out = out;
+  p.lse = lse;
+  p.q_seq = b->q_seq;
+  p.q_pos = b->q_pos;
+  p.kv_offset = b->kv_offset;
+  p.kv_len = b->kv_len;
+  p.num_seqs = b->num_seqs;
+  p.kv_rows = b->kv_rows;
+  p.T = b->num_q;
+  p.splits = mla_splits(b, k);
+  p.part_o = L.part_o;
+  p.part_lse = L.part_lse;
+  p.status = L.status;
+  return cuda_status(launch_sparse_mla(p, tq, st));
+}
+
+}  // namespace
+}  // namespace dsa
+
+using namespace dsa;
+
+extern "C" {
+
+size_t dsa_workspace_size(int op, const dsa_batch* batch, int H_I, int H, int k, int64_t ld) {
+  (void)H_I;
+  if (!batch_ok(batch)) return 0;
+  if (op < DSA_OP_INDEXER || op > DSA_OP_FORWARD) return 0;
+  if ((op == DSA_OP_SPARSE_MLA || op == DSA_OP_FORWARD) && (!h_ok(H) || !k_ok(k))) return 0;
+  if (op == DSA_OP_FORWARD && !k_ok(k)) return 0;
+  if (ld <= 0) ld = default_ld(batch);
+  return layout(nullptr, op, batch, H, k, ld).bytes;
+}
+
+dsa_status dsa_indexer_scores(const dsa_batch* batch, const uint8_t* q_idx, const uint8_t* k_idx, const float* w,
+                              int H_I, float* scores, int64_t ld, void* ws, size_t ws_bytes, void* stream) {
+  if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!q_idx || !k_idx || !w || !scores)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!hi_ok(H_I)) return DSA_ERR_UNSUPPORTED;
+  if (ld < batch->max_kv_len || ld % 4 != 0) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(scores) || !aligned16(ws))
+    return DSA_ERR_UNSUPPORTED;
+  const WsLayout L = layout(ws, DSA_OP_INDEXER, batch, 8, 1, ld);
+  if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  return run_indexer(batch, q_idx, k_idx, w, H_I, scores, ld, L, st);
+}
+
+dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t ld, int k, int32_t* idx, void* ws,
+                    size_t ws_bytes, void* stream) {
+  if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!scores || !idx)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!k_ok(k)) return DSA_ERR_UNSUPPORTED;
+  if (ld < batch->max_kv_len || ld % 4 != 0) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(scores) || !aligned16(ws)) return DSA_ERR_UNSUPPORTED;
+  const WsLayout L = layout(ws, DSA_OP_TOPK, batch, 8, k, ld);
+  if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  return run_topk(batch, scores, ld, k, idx, L, st);
+}
+
+dsa_status dsa_sparse_mla(const dsa_batch* batch, const uint16_t* q, const uint16_t* kv, const int32_t* idx, int k,
+                          int H, float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                          void* stream) {
+  if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!q || !kv || !idx || !out)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!h_ok(H) || !k_ok(k)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || !aligned16(ws)) return DSA_ERR_UNSUPPORTED;
+  const WsLayout L = layout(ws, DSA_OP_SPARSE_MLA, batch, H, k, 0);
+  if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  return run_mla(batch, q, kv, idx, k, H, sm_scale, out, lse, L, st);
+}
+
+dsa_status dsa_forward(const dsa_batch* batch, const uint8_t* q_idx, const uint8_t* k_idx, const float* w, int H_I,
+                       const uint16_t* q, const uint16_t* kv, int H, int k, float sm_scale, uint16_t* out, float* lse,
+                       void* ws, size_t ws_bytes, void* stream) {
+  if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!q_idx || !k_idx || !w || !q || !kv || !out)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!hi_ok(H_I) || !h_ok(H) || !k_ok(k)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(q) || !aligned16(kv) ||
+      !aligned16(out) || !aligned16(ws))
+    return DSA_ERR_UNSUPPORTED;
+  const int64_t ld = default_ld(batch);
+  const WsLayout L = layout(ws, DSA_OP_FORWARD, batch, H, k, ld);
+  if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  dsa_status s = run_indexer(batch, q_idx, k_idx, w, H_I, L.scores, ld, L, st);
+  if (s != DSA_OK) return s;
+  s = run_topk(batch, L.scores, ld, k, L.idx, L, st);
+  if (s != DSA_OK) return s;
+  return run_mla(batch, q, kv, L.idx, k, H, sm_scale, out, lse, L, st);
+}
+
+dsa_status dsa_forward_ws_views(const dsa_batch* batch, int H_I, int H, int k, void* ws, float** scores, int64_t* ld,
+                                int32_t** idx) {
+  (void)H_I;
+  if (!batch_ok(batch) || !ws || !scores || !ld || !idx || !h_ok(H) || !k_ok(k)) return DSA_ERR_INVALID_ARGUMENT;
+  const int64_t l = default_ld(batch);
+  const WsLayout L = layout(ws, DSA_OP_FORWARD, batch, H, k, l);
+  *scores = L.scores;
+  *ld = l;
+  *idx = L.idx;
+  return DSA_OK;
+}
+
+dsa_status dsa_read_device_status(const void* ws, uint32_t* flags, void* stream) {
+  if (!ws || !flags) return DSA_ERR_INVALID_ARGUMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  *flags = v;
+  return v == 0 ? DSA_OK : DSA_ERR_DEVICE;
+}
+
+const char* dsa_status_string(dsa_status s) {
+  switch (s) {
+    case DSA_OK: return "DSA_OK";
+    case DSA_ERR_INVALID_ARGUMENT: return "DSA_ERR_INVALID_ARGUMENT";
+    case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+    case DSA_ERR_WORKSPACE_TOO_SMALL: return "DSA_ERR_WORKSPACE_TOO_SMALL";
+    case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+    case DSA_ERR_DEVICE: return "DSA_ERR_DEVICE";
+  }
+  return "DSA_ERR_UNKNOWN";
+}
+
+int dsa_abi_version(void) { return DSA_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// Kernel parameter blocks and launchers shared between the kernels and the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace dsa {
+
+struct IndexerParams {
+  const float* w;            // [T, H_I]
+  float* scores;             // [T, ld]
+  int64_t ld;
+  const int32_t* q_seq;      // [T]
+  const int32_t* q_pos;      // [T]
+  const int64_t* kv_offset;  // [B]
+  const int32_t* kv_len;     // [B]
+  // plan (workspace)
+  int32_t* group_q0;         // [T]
+  int32_t* group_cnt;        // [T]
+  int32_t* group_seq;        // [T]
+  int32_t* group_tiles;      // [T]
+  int32_t* item_off;         // [T + 1]
+  int32_t* ngroups;          // [1]
+  int32_t* q_nvis;           // [T] visible keys per query, -1 = invalid query
+  uint32_t* status;
+  int G;                     // query tokens per group (N = G * H_I)
+  int max_kv_len;
+};
+
+struct TopkParams {
+  const float* scores;       // [T, ld]
+  int64_t ld;
+  int32_t* idx;              // [T, k]
+  int k;
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const int32_t* kv_len;
+  int num_seqs;
+  int max_kv_len;
+  uint32_t* status;
+};
+
+struct MlaParams {
+  const uint16_t* q;         // [T, H, 576] bf16
+  const uint16_t* kv;        // [rows, 576] bf16
+  const int32_t* idx;        // [T, k]
+  int k;
+  int H;
+  float sm_scale_log2;       // sm_scale * log2(e)
+  float sm_scale;
+  uint16_t* out;             // [T, H, 512] bf16
+  float* lse;                // [T, H] or null
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const int64_t* kv_offset;
+  const int32_t* kv_len;
+  int num_seqs;
+  int64_t kv_rows;
+  int T;
+  int splits;                // index-list splits per query (1 = no combine pass)
+  float* part_o;             // [T, splits, H, 512] fp32 (splits > 1)
+  float* part_lse;           // [T, splits, H]       fp32 (splits > 1)
+  uint32_t* status;
+};
+
+size_t indexer_smem_bytes();
+size_t mla_smem_bytes();
+cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int H_I,
+                           int T, int B, int64_t kv_rows, int num_sms, cudaStream_t stream);
+cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream);
+cudaError_t launch_sparse_mla(const MlaParams& p, const CUtensorMap& tm_q, cudaStream_t stream);
+
+}  // namespace dsa

@@ -1,0 +1,398 @@
+// Lightning indexer on sm_100a: I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j,:] . k_I[s,:]).
+//
+// Page "一文讀懂DeepSeek-V3.2核心技術DSA", "DSA 的四步工作流程" step 2 (indexer
+// scoring: dot products of the query against the small 128-dim key cache,
+// masked, weighted by the per-head weights); page "DeepSeek 稀疏注意力路线",
+// "两阶段流程" 1 (FP8, ReLU-type activation, aggregation over indexer heads).
+//
+// Design.  One tcgen05 GEMM per (query group, key tile):
+//   A = 128 keys of one sequence (M = 128), K-major FP8 rows of 128 B;
+//   B = G query tokens x H_I heads (N = G*H_I <= 256), K-major FP8 rows;
+//   D = fp32 [128 keys x N] in TMEM, double buffered (2 x 256 columns).
+// Keys sit in TMEM lanes, so the per-head ReLU, weighting and head sum of the
+// epilogue run along one thread's own columns with no cross-lane reduction,
+// and each warp stores 32 consecutive scores of a row (coalesced).
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..5 epilogue.  The grid is persistent (one CTA per SM); each
+// CTA takes a contiguous range of work items so the resident query tile is
+// reused across the key tiles of its group.
+#include <cstdio>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kIdxThreads = 192;
+constexpr int kKeyTile = 128;        // keys per item (MMA M)
+constexpr int kStages = 6;           // key-tile ring depth
+constexpr int kTileBytes = kKeyTile * DSA_D_INDEX;   // 16 KB
+constexpr int kQBytes = 256 * DSA_D_INDEX;           // 32 KB (N <= 256)
+
+struct __align__(8) IdxSmem {
+  uint8_t q[kQBytes];                  // 1024-aligned (offset 0)
+  uint8_t k[kStages][kTileBytes];      // 1024-aligned
+  float w[4][256];                     // per epilogue warp: head weights of the group
+  int32_t n_vis[4][256];               // per epilogue warp: visible keys per token
+  uint64_t k_full[kStages], k_empty[kStages];
+  uint64_t q_full, q_empty;
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Largest g with item_off[g] <= i (item_off is non-decreasing, item_off[0] = 0).
+__device__ __forceinline__ int find_group(const int32_t* item_off, int ngroups, int i) {
+  int lo = 0, hi = ngroups - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (item_off[mid] <= i) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int HI>
+__global__ void __launch_bounds__(kIdxThreads, 1)
+indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               IndexerParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  IdxSmem& S = *reinterpret_cast<IdxSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ngroups = *p.ngroups;
+  const int total = ngroups > 0 ? p.item_off[ngroups] : 0;
+  const int per = (total + gridDim.x - 1) / gridDim.x;
+  const int i0 = min(total, static_cast<int>(blockIdx.x) * per);
+  const int i1 = min(total, i0 + per);
+  const int N = p.G * HI;
+  volatile int* abort_flag = &S.abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&S.k_full[s], 1); mbar_init(&S.k_empty[s], 1); }
+    mbar_init(&S.q_full, 1);
+    mbar_init(&S.q_empty, 1);
+    for (int a = 0; a < 2; ++a) { mbar_init(&S.acc_full[a], 1); mbar_init(&S.acc_empty[a], 128); }
+    mbar_init(&S.done, 1);
+    S.abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+  }
+  if (warp == 1) tmem_alloc(&S.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+
+  if (i0 < i1) {
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        int g = find_group(p.item_off, ngroups, i0);
+        int prev_g = -1, issued = 0, q_loads = 0;
+        uint32_t qe_par = 0;
+        for (int i = i0; i < i1; ++i) {
+          while (p.item_off[g + 1] <= i) ++g;
+          const int kt = i - p.item_off[g];
+          if (g != prev_g) {
+            if (prev_g >= 0) {
+              if (!mbar_wait(&S.q_empty, qe_par, p.status, abort_flag)) break;
+              qe_par ^= 1;
+            }
+            mbar_arrive_expect_tx(&S.q_full, N * DSA_D_INDEX);
+            tma_load_2d(S.q, &tm_q, &S.q_full, 0, p.group_q0[g] * HI);
+            ++q_loads;
+            prev_g = g;
+          }
+          const int n = i - i0, st = n % kStages;
+          const uint32_t ph = (n / kStages) & 1;
+          if (!mbar_wait(&S.k_empty[st], ph ^ 1, p.status, abort_flag)) break;
+          mbar_arrive_expect_tx(&S.k_full[st], kTileBytes);
+          const int64_t row = p.kv_offset[p.group_seq[g]] + static_cast<int64_t>(kt) * kKeyTile;
+          tma_load_2d(S.k[st], &tm_k, &S.k_full[st], 0, static_cast<int>(row));
+          ++issued;
+        }
+        // Never leave with a copy in flight: wait (bounded) for the last load of each stage.
+        for (int n = max(0, issued - kStages); n < issued; ++n)
+          mbar_wait(&S.k_full[n % kStages], (n / kStages) & 1, p.status, nullptr);
+        if (q_loads > 0) mbar_wait(&S.q_full, (q_loads - 1) & 1, p.status, nullptr);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc = instr_desc(0, 0, false, false, kKeyTile, N);
+        int g = find_group(p.item_off, ngroups, i0);
+        int prev_g = -1;
+        uint32_t qf_par = 0;
+        for (int i = i0; i < i1; ++i) {
+          while (p.item_off[g + 1] <= i) ++g;
+          if (g != prev_g) {
+            if (!mbar_wait(&S.q_full, qf_par, p.status, abort_flag)) break;
+            qf_par ^= 1;
+            prev_g = g;
+          }
+          const int n = i - i0, st = n % kStages, a = n & 1;
+          const uint32_t ph = (n / kStages) & 1, aph = (n >> 1) & 1;
+          if (!mbar_wait(&S.acc_empty[a], aph ^ 1, p.status, abort_flag)) break;
+          tc_fence_after();
+          if (!mbar_wait(&S.k_full[st], ph, p.status, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(S.k[st]);
+          const uint32_t b_base = smem_u32(S.q);
+          const uint32_t d = tmem + a * 256;
+#pragma unroll
+          for (int kk = 0; kk < DSA_D_INDEX / 32; ++kk) {
+            const uint64_t ad = smem_desc_sw128(a_base + kk * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+            umma_f8(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&S.k_empty[st]);
+          umma_commit(&S.acc_full[a]);
+          const bool last_of_group = (i + 1 == i1) || (p.item_off[g + 1] <= i + 1);
+          if (last_of_group) umma_commit(&S.q_empty);
+        }
+        umma_commit(&S.done);
+        mbar_wait(&S.done, 0, p.status, nullptr);
+      }
+    } else {
+      // ------------------------------------------------------------ epilogue
+      // Warp-uniform control flow: lane 0 waits on barriers, the warp follows.
+      const int quad = warp & 3;                  // TMEM lane quadrant of this warp
+      const int row = quad * 32 + lane;           // key within the tile
+      float* sw = S.w[warp - 2];
+      int32_t* snv = S.n_vis[warp - 2];
+      int g = find_group(p.item_off, ngroups, i0);
+      int prev_g = -1, cnt = 0, q0 = 0;
+      for (int i = i0; i < i1; ++i) {
+        while (p.item_off[g + 1] <= i) ++g;
+        const int kt = i - p.item_off[g];
+        if (g != prev_g) {
+          __syncwarp();
+          q0 = p.group_q0[g];
+          cnt = p.group_cnt[g];
+          for (int j = lane; j < cnt * HI; j += 32) sw[j] = p.w[static_cast<int64_t>(q0) * HI + j];
+          for (int j = lane; j < cnt; j += 32) snv[j] = max(0, p.q_nvis[q0 + j]);
+          __syncwarp();
+          prev_g = g;
+        }
+        const int n = i - i0, a = n & 1;
+        const uint32_t aph = (n >> 1) & 1;
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&S.acc_full[a], aph, p.status, abort_flag) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+        const int s = kt * kKeyTile + row;
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + a * 256;
+        if constexpr (HI >= 32) {
+          for (int tok = 0; tok < cnt; ++tok) {
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < HI / 32; ++c) {
+              uint32_t v[32];
+              tmem_ld32(tbase + tok * HI + c * 32, v);
+              tmem_ld_wait();
+              const float* wr = &sw[tok * HI + c * 32];
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) {
+                const float4 w4 = *reinterpret_cast<const float4*>(wr + j);
+                acc = fmaf(w4.x, fmaxf(__uint_as_float(v[j + 0]), 0.f), acc);
+                acc = fmaf(w4.y, fmaxf(__uint_as_float(v[j + 1]), 0.f), acc);
+                acc = fmaf(w4.z, fmaxf(__uint_as_float(v[j + 2]), 0.f), acc);
+                acc = fmaf(w4.w, fmaxf(__uint_as_float(v[j + 3]), 0.f), acc);
+              }
+            }
+            if (s < snv[tok]) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = acc;
+          }
+        } else {
+          constexpr int TPC = 32 / HI;             // tokens per 32-column chunk
+          const int nchunks = (cnt * HI + 31) / 32;
+          for (int c = 0; c < nchunks; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tbase + c * 32, v);
+            tmem_ld_wait();
+            float acc[TPC];
+#pragma unroll
+            for (int u = 0; u < TPC; ++u) acc[u] = 0.f;
+            const float* wr = &sw[c * 32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              acc[j / HI] = fmaf(wr[j], fmaxf(__uint_as_float(v[j]), 0.f), acc[j / HI]);
+            }
+#pragma unroll
+            for (int u = 0; u < TPC; ++u) {
+              const int tok = c * TPC + u;
+              if (tok < cnt && s < snv[tok]) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = acc[u];
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&S.acc_empty[a]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------------- planning
+// One CTA.  Forms groups of at most G consecutive queries of one sequence,
+// records each group's first query, size and sequence, the number of 128-key
+// tiles its last query needs, and the exclusive prefix of those counts.
+constexpr int kPlanThreads = 1024;
+
+__device__ int block_inclusive_scan(int v, int* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += x;
+  }
+  if (lane == 31) scratch[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < (blockDim.x >> 5) ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += x;
+    }
+    scratch[lane] = t;
+  }
+  __syncthreads();
+  if (warp > 0) v += scratch[warp - 1];
+  __syncthreads();
+  return v;
+}
+
+// Visible keys of query t (q_pos + 1), or -1 when its sequence or position is
+// out of range (the query then gets no scores).
+__device__ __forceinline__ int visible_keys(const IndexerParams& p, int t, int B, int64_t kv_rows) {
+  const int seq = p.q_seq[t];
+  if (seq < 0 || seq >= B) return -1;
+  const int len = p.kv_len[seq];
+  const int64_t off = p.kv_offset[seq];
+  const int pos = p.q_pos[t];
+  if (len < 0 || len > p.max_kv_len || off < 0 || off + len > kv_rows || pos < 0 || pos >= len) return -1;
+  return pos + 1;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) indexer_plan_kernel(IndexerParams p, int T, int B, int64_t kv_rows) {
+  __shared__ int scratch[32];
+  __shared__ int carry_groups, carry_run_start, carry_tiles;
+  if (threadIdx.x == 0) { carry_groups = 0; carry_run_start = 0; carry_tiles = 0; }
+  __syncthreads();
+  // Pass 1: leaders and group records.
+  for (int base = 0; base < T; base += kPlanThreads) {
+    const int t = base + threadIdx.x;
+    int seq = -1;
+    bool run_start = false;
+    if (t < T) {
+      seq = p.q_seq[t];
+      run_start = (t == 0) || (p.q_seq[t - 1] != seq);
+      const int nv = visible_keys(p, t, B, kv_rows);
+      p.q_nvis[t] = nv;
+      if (nv < 0) set_status(p.status, DSA_DEV_BAD_QUERY);
+    }
+    // last run start at or before t: inclusive max-scan of (run_start ? t : -1)
+    int rs = run_start ? t : -1;
+    {
+      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, rs, o);
+        if (lane >= o) rs = max(rs, x);
+      }
+      if (lane == 31) scratch[warp] = rs;
+      __syncthreads();
+      if (warp == 0) {
+        int m = scratch[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int x = __shfl_up_sync(0xffffffffu, m, o);
+          if (lane >= o) m = max(m, x);
+        }
+        scratch[lane] = m;
+      }
+      __syncthreads();
+      if (warp > 0) rs = max(rs, scratch[warp - 1]);
+      rs = max(rs, carry_run_start);
+      __syncthreads();
+    }
+    const bool leader = (t < T) && (((t - rs) % p.G) == 0);
+    const int inc = block_inclusive_scan(leader ? 1 : 0, scratch);
+    if (leader) {
+      const int gi = carry_groups + inc - 1;
+      int cnt = 1, maxn = 0;
+      for (int u = 0; u < p.G && t + u < T; ++u) {
+        const int tu = t + u;
+        if (u > 0 && p.q_seq[tu] != seq) break;
+        cnt = u + 1;
+        maxn = max(maxn, max(0, visible_keys(p, tu, B, kv_rows)));
+      }
+      p.group_q0[gi] = t;
+      p.group_cnt[gi] = cnt;
+      p.group_seq[gi] = (seq >= 0 && seq < B) ? seq : 0;
+      p.group_tiles[gi] = (maxn + kKeyTile - 1) / kKeyTile;
+    }
+    __syncthreads();
+    if (threadIdx.x == kPlanThreads - 1) {
+      carry_groups += inc;
+      carry_run_start = max(carry_run_start, rs);
+    }
+    __syncthreads();
+  }
+  const int ngroups = carry_groups;
+  // Pass 2: exclusive prefix of tile counts.
+  for (int base = 0; base < ngroups; base += kPlanThreads) {
+    const int gi = base + threadIdx.x;
+    const int v = gi < ngroups ? p.group_tiles[gi] : 0;
+    const int inc = block_inclusive_scan(v, scratch);
+    if (gi < ngroups) p.item_off[gi] = carry_tiles + inc - v;
+    __syncthreads();
+    if (threadIdx.x == kPlanThreads - 1) carry_tiles += inc;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    p.item_off[ngroups] = carry_tiles;
+    *p.ngroups = ngroups;
+  }
+}
+
+}  // namespace
+
+size_t indexer_smem_bytes() { return sizeof(IdxSmem) + 1024; }
+
+cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int H_I,
+                           int T, int B, int64_t kv_rows, int num_sms, cudaStream_t stream) {
+  indexer_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p, T, B, kv_rows);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = indexer_smem_bytes();
+  auto launch = [&](auto kern) -> cudaError_t {
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    kern<<<num_sms, kIdxThreads, smem, stream>>>(tm_q, tm_k, p);
+    return cudaGetLastError();
+  };
+  switch (H_I) {
+    case 4: return launch(indexer_kernel<4>);
+    case 8: return launch(indexer_kernel<8>);
+    case 16: return launch(indexer_kernel<16>);
+    case 32: return launch(indexer_kernel<32>);
+    case 64: return launch(indexer_kernel<64>);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace dsa

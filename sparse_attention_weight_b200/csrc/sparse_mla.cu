@@ -1,0 +1,510 @@
+// Sparse MLA in MQA form on sm_100a.
+//
+// Page "一文讀懂DeepSeek-V3.2核心技術DSA", "DSA 的四步工作流程" step 4: attention
+// over only the selected tokens; page "DeepSeek-V3.2加速技术详解" 3.1 (MQA form of
+// MLA: every head attends to the shared latent row, the value is the latent,
+// restored afterwards) and 3.2 (unselected tokens are dropped); page "DeepSeek
+// 稀疏注意力路线", "工程要点" (the top-k index list makes the KV gather irregular).
+//
+// Per query token the state is large: Q is 128 heads x 576 (144 KB bf16) and
+// the output accumulator 128 x 512 fp32 (256 KB, all of one SM's TMEM).  So a
+// token is handled by a CTA pair (a 2-CTA cluster) using the pair form of the
+// tensor-core MMA (cta_group::2, M = 128 = 64 heads per CTA):
+//   S  = Q K^T : A = the CTA's 64 heads of Q (72 KB, resident), B = a block of
+//                128 gathered rows, split 64/64 between the CTAs (K-major);
+//                per CTA: 64 heads x 128 rows fp32 in TMEM (64 columns).
+//   O += P V   : A = P (64 heads x 128 rows, bf16, written by the softmax
+//                warps), B = V rows of the block, each CTA holding 128 of every
+//                256 value dims (MN-major); per CTA: 64 heads x 512 dims fp32
+//                (256 TMEM columns).
+// S is double buffered in TMEM, so the tensor core computes S of block j+1
+// while the softmax warps turn S of block j into P.  The softmax keeps a
+// reference maximum per head and rescales O (in TMEM) only when a block's
+// maximum exceeds it by more than 2^8, so P stays <= 256 and most blocks skip
+// the rescale.  Rows are gathered by index with 16-byte cp.async (8 lanes per
+// 128-byte row segment: coalesced) into 128-byte-swizzled tiles.
+//
+// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-5 gather of the
+// S operand rows, 6-7 gather of the V operand rows, 8 TMEM owner and (in the
+// even CTA) MMA issuer.
+#include <cuda_bf16.h>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kMlaThreads = 288;
+constexpr int kBlk = 128;             // selected rows per block (pair)
+constexpr int kHalf = 64;             // rows per CTA for the S operand; heads per CTA
+constexpr int kDChunks = DSA_D_QK / 64;   // 9 chunks of 64 dims
+constexpr int kSStages = 8;           // S-operand ring (8 KB slots)
+constexpr int kVStages = 6;           // V-operand ring (8 KB slots)
+constexpr int kLag = 3;               // cp.async groups kept in flight per producer thread
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr uint32_t kSCol = 0;         // TMEM columns [0,128): two S buffers of 64
+constexpr uint32_t kOCol = 128;       // TMEM columns [128,384): O (2 x 128)
+
+struct __align__(1024) MlaSmem {
+  uint8_t q[kDChunks][kHalf * 128];          // 72 KB  Q of this CTA's heads (K-major SW128)
+  uint8_t s_ring[kSStages][kHalf * 128];     // 64 KB  S operand chunks: 64 rows x 64 dims
+  uint8_t v_ring[kVStages][4][16 * 128];     // 48 KB  V operand chunks: 16 rows x 4 dim groups
+  uint8_t p[2][kHalf * 128];                 // 16 KB  P: 64 heads x 128 rows (two K chunks)
+  float xmax[2][128];
+  float lsum[128];
+  uint64_t q_full, q_ready;
+  uint64_t s_full[kSStages], s_empty[kSStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_ready[2], s_free[2];
+  uint64_t p_full, p_empty;
+  uint64_t mx_bar[2], l_bar;
+  uint64_t done;
+  uint32_t tmem_base;
+  int nblk, blk0;
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Lane-0 waits, the warp follows (warp-uniform result).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* status, volatile int* ab,
+                                          bool cluster_scope) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0)
+    ok = (cluster_scope ? mbar_wait_cluster(bar, parity, status, ab) : mbar_wait(bar, parity, status, ab)) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Global row of selected entry `pos` of query t, or -1 when unused/invalid.
+__device__ __forceinline__ int64_t sel_row(const MlaParams& p, const int32_t* idx_row, int pos, int64_t base,
+                                           int len) {
+  if (pos >= p.k) return -1;
+  const int i = __ldg(idx_row + pos);
+  if (i < 0) return -1;
+  if (i >= len) { set_status(p.status, DSA_DEV_BAD_INDEX); return -1; }
+  return base + i;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
+sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  MlaSmem& S = *reinterpret_cast<MlaSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int cid = blockIdx.x >> 1;
+  const int t = cid / p.splits;
+  const int split = cid % p.splits;
+  volatile int* ab = &S.abort_flag;
+
+  // ---- per-query facts (identical in both CTAs)
+  const int seq = p.q_seq[t];
+  const bool seq_ok = seq >= 0 && seq < p.num_seqs;
+  const int len = seq_ok ? p.kv_len[seq] : 0;
+  const int64_t base = seq_ok ? p.kv_offset[seq] : 0;
+  const bool rows_ok = seq_ok && len >= 0 && base >= 0 && base + len <= p.kv_rows;
+  const int32_t* idx_row = p.idx + static_cast<int64_t>(t) * p.k;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&S.q_full, 1);
+    mbar_init(&S.q_ready, 2);
+    for (int i = 0; i < kSStages; ++i) { mbar_init(&S.s_full[i], 4); mbar_init(&S.s_empty[i], 1); }
+    for (int i = 0; i < kVStages; ++i) { mbar_init(&S.v_full[i], 4); mbar_init(&S.v_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 8); mbar_init(&S.mx_bar[i], 128);
+    }
+    mbar_init(&S.p_full, 8);
+    mbar_init(&S.p_empty, 1);
+    mbar_init(&S.l_bar, 128);
+    mbar_init(&S.done, 1);
+    S.abort_flag = 0;
+    fence_mbar_init();
+    if (!rows_ok) set_status(p.status, DSA_DEV_BAD_QUERY);
+  }
+  // blocks of 128 entries covering the used part of the index row, split evenly
+  if (warp == 4) {
+    int last = -1;
+    if (rows_ok) {
+      for (int i = lane; i < p.k; i += 32)
+        if (__ldg(idx_row + i) >= 0) last = i;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+    if (lane == 0) {
+      const int total = (last + kBlk) / kBlk;
+      const int per = (total + p.splits - 1) / p.splits;
+      const int b0 = min(total, split * per);
+      S.blk0 = b0;
+      S.nblk = min(total, b0 + per) - b0;
+    }
+  }
+  if (warp == 8) tmem_alloc_pair(&S.tmem_base, 512);
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  const int nblk = S.nblk;
+  const int blk0 = S.blk0;
+
+  const int H = p.H;
+  const int head0 = static_cast<int>(rank) * kHalf;        // first head of this CTA
+
+  if (nblk > 0) {
+    if (warp < 4) {
+      // ================================================================ softmax
+      const int tid = threadIdx.x;                           // TMEM lane
+      const int hl = tid & 63;                               // local head
+      const int half = tid >> 6;                             // which 64 rows of each block
+      const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < nblk; ++j) {
+        const int sb = j & 1;
+        const uint32_t sph = (j >> 1) & 1;
+        // validity of this warp's 64 columns
+        const int pos0 = (blk0 + j) * kBlk + half * 64;
+        uint32_t vm0, vm1;
+        {
+          const int pa = pos0 + lane, pb = pos0 + 32 + lane;
+          const bool va = pa < p.k && __ldg(idx_row + pa) >= 0 && __ldg(idx_row + pa) < len;
+          const bool vb = pb < p.k && __ldg(idx_row + pb) >= 0 && __ldg(idx_row + pb) < len;
+          vm0 = __ballot_sync(0xffffffffu, va);
+          vm1 = __ballot_sync(0xffffffffu, vb);
+        }
+        if (!warp_wait(&S.s_ready[sb], sph, p.status, ab, false)) break;
+        tc_fence_after();
+        uint32_t sr[64];
+        {
+          uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+          uint32_t (&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+          tmem_ld32(tmem + lane_addr + kSCol + sb * 64, a);
+          tmem_ld32(tmem + lane_addr + kSCol + sb * 64 + 32, b);
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(&S.s_free[sb], 0);
+        float* x = reinterpret_cast<float*>(sr);             // logits in log2 units, in place
+        float mloc = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const bool v = ((c < 32 ? vm0 >> c : vm1 >> (c - 32)) & 1u) != 0;
+          x[c] = v ? __uint_as_float(sr[c]) * p.sm_scale_log2 : -INFINITY;
+          mloc = fmaxf(mloc, x[c]);
+        }
+        // pair maximum of this head over the whole block
+        S.xmax[sb][tid] = mloc;
+        mbar_arrive(&S.mx_bar[sb]);
+        if (!warp_wait(&S.mx_bar[sb], sph, p.status, ab, false)) break;
+        const float mblk = fmaxf(mloc, S.xmax[sb][tid ^ 64]);
+        const bool rescale = mblk > m_ref + kRescaleThreshold;
+        const float m_new = rescale ? mblk : m_ref;
+        float psum = 0.f;
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = x[c] == -INFINITY ? 0.f : exp2f(x[c] - m_new);
+          const float p1 = x[c + 1] == -INFINITY ? 0.f : exp2f(x[c + 1] - m_new);
+          psum += p0 + p1;
+          pk[c >> 1] = pack_bf16(p0, p1);
+        }
+        const float alpha = rescale ? exp2f(m_ref - m_new) : 1.f;   // m_ref = -inf -> 0
+        l = l * alpha + psum;
+        // P buffer and O are free once PV of the previous block completed
+        if (j > 0) {
+          if (!warp_wait(&S.p_empty, (j - 1) & 1, p.status, ab, false)) break;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, rescale)) {   // TMEM ld/st are warp-collective
+#pragma unroll 1
+            for (int c = 0; c < 16; ++c) {
+              uint32_t o[16];
+              const uint32_t a = tmem + lane_addr + kOCol + c * 16;
+              tmem_ld16(a, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+              tmem_st16(a, o);
+            }
+            tmem_st_wait();
+          }
+        }
+        m_ref = m_new;
+        // P row hl, K chunk `half` (rows half*64 .. +63 of the block), 128B-swizzled
+        {
+          uint8_t* prow = S.p[half] + hl * 128;
+#pragma unroll
+          for (int c16 = 0; c16 < 8; ++c16) {
+            const uint32_t off = static_cast<uint32_t>(((c16 ^ (hl & 7)) << 4));
+            *reinterpret_cast<uint4*>(prow + off) =
+                make_uint4(pk[c16 * 4 + 0], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(&S.p_full, 0);
+      }
+      // ---- epilogue: wait for the last PV, combine the two row halves, write out
+      bool ok = !*ab;
+      if (ok) ok = warp_wait(&S.p_empty, (nblk - 1) & 1, p.status, ab, false);
+      if (ok) {
+        tc_fence_after();
+        S.lsum[tid] = l;
+        mbar_arrive(&S.l_bar);
+        ok = warp_wait(&S.l_bar, 0, p.status, ab, false);
+      }
+      if (ok) {
+        const float lt = l + S.lsum[tid ^ 64];
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const int h = head0 + hl;
+        const bool store = h < H;                            // TMEM loads stay warp-collective
+        const float lse_v = lt > 0.f ? (m_ref + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        if (p.splits == 1) {
+          uint16_t* orow = p.out + (static_cast<int64_t>(t) * H + (store ? h : 0)) * DSA_D_V;
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tmem + lane_addr + kOCol + c * 16, o);
+            tmem_ld_wait();
+            const int d0 = (c >> 3) * 256 + half * 128 + (c & 7) * 16;
+            uint32_t pkd[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              pkd[u] = pack_bf16(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv);
+            if (store) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + d0);
+              dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+              dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+            }
+          }
+          if (store && half == 0 && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = lse_v;
+        } else {
+          float* orow = p.part_o + ((static_cast<int64_t>(t) * p.splits + split) * H + (store ? h : 0)) * DSA_D_V;
+#pragma unroll 1
+          for (int c = 0; c < 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tmem + lane_addr + kOCol + c * 16, o);
+            tmem_ld_wait();
+            const int d0 = (c >> 3) * 256 + half * 128 + (c & 7) * 16;
+            if (store) {
+              float4* dst = reinterpret_cast<float4*>(orow + d0);
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                dst[u] = make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
+                                     __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
+            }
+          }
+          if (store && half == 0)
+            p.part_lse[(static_cast<int64_t>(t) * p.splits + split) * H + h] = lse_v;
+        }
+      }
+    } else if (warp < 6) {
+      // ================================================================ S-operand gather
+      const int pt = threadIdx.x - 128;                      // 0..63
+      const int c16 = pt & 7;
+      if (threadIdx.x == 128) {
+        // this CTA's 64 heads of Q: 9 TMA boxes of 64 dims x 64 rows
+        mbar_arrive_expect_tx(&S.q_full, kDChunks * kHalf * 128);
+        for (int dc = 0; dc < kDChunks; ++dc)
+          tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
+        if (mbar_wait(&S.q_full, 0, p.status, ab)) mbar_arrive_cluster(&S.q_ready, 0);
+      }
+      const int nchunks = nblk * kDChunks;
+      for (int n = 0; n < nchunks + kLag; ++n) {
+        if (n < nchunks) {
+          const int j = n / kDChunks, dc = n % kDChunks, st = n % kSStages;
+          if (!warp_wait(&S.s_empty[st], ((n / kSStages) & 1) ^ 1, p.status, ab, false)) break;
+          const uint32_t dst0 = smem_u32(S.s_ring[st]);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int r = it * 8 + (pt >> 3);                  // row within this CTA's 64
+            const int64_t g = sel_row(p, idx_row, (blk0 + j) * kBlk + static_cast<int>(rank) * kHalf + r, base, len);
+            const uint16_t* src = p.kv + (g < 0 ? 0 : g) * DSA_D_QK + dc * 64 + c16 * 8;
+            cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4), src, g < 0 ? 0u : 16u);
+          }
+        }
+        cp_async_commit();
+        if (n >= kLag) {
+          cp_async_wait<kLag>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(&S.s_full[(n - kLag) % kSStages], 0);
+        }
+      }
+      cp_async_wait<0>();
+    } else if (warp < 8) {
+      // ================================================================ V-operand gather
+      const int pt = threadIdx.x - 192;                      // 0..63
+      const int c16 = pt & 7;
+      const int nchunks = nblk * (kBlk / 16);
+      for (int n = 0; n < nchunks + kLag; ++n) {
+        if (n < nchunks) {
+          const int j = n / (kBlk / 16), kk = n % (kBlk / 16), st = n % kVStages;
+          if (!warp_wait(&S.v_empty[st], ((n / kVStages) & 1) ^ 1, p.status, ab, false)) break;
+          const uint32_t dst0 = smem_u32(S.v_ring[st]);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int pi = it * 8 + (pt >> 3);                 // (row, group) pair 0..63
+            const int r = pi & 15, grp = pi >> 4;
+            const int d0 = (grp >> 1) * 256 + static_cast<int>(rank) * 128 + (grp & 1) * 64;
+            const int64_t g = sel_row(p, idx_row, (blk0 + j) * kBlk + kk * 16 + r, base, len);
+            const uint16_t* src = p.kv + (g < 0 ? 0 : g) * DSA_D_QK + d0 + c16 * 8;
+            cp_async16(dst0 + grp * 2048 + r * 128 + ((c16 ^ (r & 7)) << 4), src, g < 0 ? 0u : 16u);
+          }
+        }
+        cp_async_commit();
+        if (n >= kLag) {
+          cp_async_wait<kLag>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(&S.v_full[(n - kLag) % kVStages], 0);
+        }
+      }
+      cp_async_wait<0>();
+    } else if (rank == 0 && lane == 0) {
+      // ================================================================ MMA issuer (even CTA)
+      const uint32_t id_s = instr_desc(1, 1, false, false, 128, kBlk);   // bf16 x bf16, M=128 pair, N=128
+      const uint32_t id_pv = instr_desc(1, 1, false, true, 128, 256);    // B (V) MN-major, N=256
+      bool ok = mbar_wait_cluster(&S.q_ready, 0, p.status, ab);
+      int sc = 0, vc = 0;
+      auto issue_s = [&](int j) -> bool {
+        const int sb = j & 1;
+        if (!mbar_wait_cluster(&S.s_free[sb], ((j >> 1) & 1) ^ 1, p.status, ab)) return false;
+        tc_fence_after();
+        for (int dc = 0; dc < kDChunks; ++dc, ++sc) {
+          const int st = sc % kSStages;
+          if (!mbar_wait_cluster(&S.s_full[st], (sc / kSStages) & 1, p.status, ab)) return false;
+          tc_fence_after();
+          const uint32_t qa = smem_u32(S.q[dc]);
+          const uint32_t sa = smem_u32(S.s_ring[st]);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_pair(tmem + kSCol + sb * 64, smem_desc_sw128(qa + kk * 32, 16, 1024),
+                           smem_desc_sw128(sa + kk * 32, 16, 1024), id_s, (dc | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(&S.s_empty[st], 0x3);
+        }
+        umma_commit_pair(&S.s_ready[sb], 0x3);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        if (!mbar_wait_cluster(&S.p_full, j & 1, p.status, ab)) return false;
+        tc_fence_after();
+        for (int kk = 0; kk < kBlk / 16; ++kk, ++vc) {
+          const int st = vc % kVStages;
+          if (!mbar_wait_cluster(&S.v_full[st], (vc / kVStages) & 1, p.status, ab)) return false;
+          tc_fence_after();
+          const uint32_t pa = smem_u32(S.p[kk >> 2]) + (kk & 3) * 32;
+          const uint32_t va = smem_u32(S.v_ring[st]);
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            umma_bf16_pair(tmem + kOCol + c * 128, smem_desc_sw128(pa, 16, 1024),
+                           smem_desc_sw128(va + c * 4096, 2048, 1024), id_pv, (j | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(&S.v_empty[st], 0x3);
+        }
+        umma_commit_pair(&S.p_empty, 0x3);
+        return true;
+      };
+      if (ok) {
+        for (int j = 0; j < nblk && ok; ++j) {
+          ok = issue_s(j);
+          if (ok && j >= 1) ok = issue_pv(j - 1);
+        }
+        if (ok) ok = issue_pv(nblk - 1);
+      }
+      umma_commit_pair(&S.done, 0x1);                       // drain: every MMA of this pair completed
+      mbar_wait(&S.done, 0, p.status, nullptr);
+    }
+  } else if (warp < 4) {
+    // no selected row: output zeros, lse = -inf
+    const int tid = threadIdx.x;
+    const int hl = tid & 63, half = tid >> 6;
+    const int h = head0 + hl;
+    if (h < H) {
+      if (p.splits == 1) {
+        uint16_t* orow = p.out + (static_cast<int64_t>(t) * H + h) * DSA_D_V;
+        for (int d = half * 256; d < half * 256 + 256; d += 8)
+          *reinterpret_cast<uint4*>(orow + d) = make_uint4(0, 0, 0, 0);
+        if (half == 0 && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = -INFINITY;
+      } else {
+        float* orow = p.part_o + ((static_cast<int64_t>(t) * p.splits + split) * H + h) * DSA_D_V;
+        for (int d = half * 256; d < half * 256 + 256; d += 4)
+          *reinterpret_cast<float4*>(orow + d) = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (half == 0) p.part_lse[(static_cast<int64_t>(t) * p.splits + split) * H + h] = -INFINITY;
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+// Merge split partial results: lse = log sum exp(lse_i); out = sum exp(lse_i - lse) o_i.
+__global__ void __launch_bounds__(128) mla_combine_kernel(MlaParams p) {
+  const int t = blockIdx.x, h = blockIdx.y;
+  const int64_t pr = (static_cast<int64_t>(t) * p.splits) * p.H + h;
+  float mx = -INFINITY;
+  for (int s = 0; s < p.splits; ++s) mx = fmaxf(mx, p.part_lse[pr + static_cast<int64_t>(s) * p.H]);
+  float den = 0.f;
+  for (int s = 0; s < p.splits; ++s) {
+    const float ls = p.part_lse[pr + static_cast<int64_t>(s) * p.H];
+    den += ls == -INFINITY ? 0.f : __expf(ls - mx);
+  }
+  const int d = threadIdx.x * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < p.splits; ++s) {
+    const float ls = p.part_lse[pr + static_cast<int64_t>(s) * p.H];
+    if (ls == -INFINITY) continue;
+    const float wgt = __expf(ls - mx) / den;
+    const float4 o = *reinterpret_cast<const float4*>(p.part_o + (pr + static_cast<int64_t>(s) * p.H) * DSA_D_V + d);
+    acc.x += wgt * o.x; acc.y += wgt * o.y; acc.z += wgt * o.z; acc.w += wgt * o.w;
+  }
+  uint16_t* orow = p.out + (static_cast<int64_t>(t) * p.H + h) * DSA_D_V + d;
+  *reinterpret_cast<uint2*>(orow) = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+  if (threadIdx.x == 0 && p.lse)
+    p.lse[static_cast<int64_t>(t) * p.H + h] = den > 0.f ? mx + __logf(den) : -INFINITY;
+}
+
+}  // namespace
+
+size_t mla_smem_bytes() { return sizeof(MlaSmem) + 1024; }
+
+cudaError_t launch_sparse_mla(const MlaParams& p, const CUtensorMap& tm_q, cudaStream_t stream) {
+  if (p.T == 0) return cudaSuccess;
+  const size_t smem = mla_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  sparse_mla_kernel<<<2 * p.T * p.splits, kMlaThreads, smem, stream>>>(tm_q, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.splits == 1) return e;
+  mla_combine_kernel<<<dim3(p.T, p.H), 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

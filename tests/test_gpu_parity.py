@@ -1,0 +1,311 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Same seeded inputs on both sides.  Bars: top-k bit-exact given the oracle's
+scores (rounded to fp32); indexer scores within 1e-4 of max(|I|, sum|w|ReLU);
+attention outputs within max-abs 1e-2 / mean-abs 1e-3 of the fp64 oracle;
+end to end, selection mismatches only where scores tie the k-th score to 1e-4.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_weight_b200 import binding as B
+from sparse_attention_weight_b200 import build, inputs
+from sparse_attention_weight_b200.configs import WORKLOADS, Workload
+
+from . import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+MID_PREFILL = Workload("mid_prefill", 20, "prefill", k=2048, h_index=64, heads=128, seq_len=2600)
+MID_DEC2 = Workload("mid_decode2", 21, "decode", k=2048, h_index=64, heads=128, batch=6, ctx_min=1500,
+                    ctx_max=5000, q_per_seq=2)
+MID_DEC1 = Workload("mid_decode1", 22, "decode", k=512, h_index=64, heads=128, batch=5, ctx_min=300,
+                    ctx_max=3000, q_per_seq=1)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+    B.lib()
+
+
+def _sample_rows(T, k, extra=()):
+    rows = {0, 1, T - 1, T - 2, min(T - 1, k - 1), min(T - 1, k), min(T - 1, k + 1), min(T - 1, 127),
+            min(T - 1, 128), T // 2}
+    rows |= set(int(x) for x in extra)
+    rng = np.random.default_rng(123)
+    rows |= set(int(x) for x in rng.integers(0, T, size=12))
+    return sorted(r for r in rows if 0 <= r < T)
+
+
+def _run_indexer(dev, wl, batch_host):
+    T = batch_host.num_q
+    ld = (batch_host.max_kv_len + 3) // 4 * 4
+    scores = torch.full((T, ld), float("nan"), device=dev)
+    ws = B.workspace(B.OP_INDEXER, dev["batch"], H_I=wl.h_index, ld=ld, device=scores.device)
+    B.dsa_indexer_scores(dev["batch"], dev["q_idx"], dev["k_idx"], dev["w"], wl.h_index, scores, ld, ws)
+    assert B.read_device_status(ws) == 0
+    return scores.cpu().numpy()
+
+
+# ----------------------------------------------------------------------------- indexer
+
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny_prefill"], MID_PREFILL, MID_DEC2, MID_DEC1,
+                                Workload("hi8", 23, "prefill", k=64, h_index=8, heads=8, seq_len=700),
+                                Workload("hi16", 24, "prefill", k=64, h_index=16, heads=8, seq_len=700),
+                                Workload("hi32", 25, "prefill", k=64, h_index=32, heads=8, seq_len=700)],
+                         ids=lambda w: w.name)
+def test_indexer_scores_match_oracle(cuda_device, wl):
+    ins = inputs.make_inputs(wl)
+    batch = ins["batch"]
+    dev = H.to_device(ins, cuda_device)
+    got = _run_indexer(dev, wl, batch)
+    T = batch.num_q
+    rows = range(T) if T <= 1100 else _sample_rows(T, wl.k)
+    for t in rows:
+        I, A = H.indexer_ref_row(ins, t)
+        n = int(batch.q_pos[t]) + 1
+        H.check_indexer_row(got[t, :n], I, A, f"{wl.name} row {t}")
+        # nothing written beyond the visible keys
+        assert np.isnan(got[t, n:]).all()
+
+# ----------------------------------------------------------------------------- top-k
+
+
+def _topk_case(cuda_device, rows, k):
+    """rows: list of float32 arrays (row t has n_t = len(rows[t]))."""
+    T = len(rows)
+    nmax = max(len(r) for r in rows)
+    ld = (nmax + 3) // 4 * 4
+    sc = np.full((T, ld), np.nan, np.float32)
+    for t, r in enumerate(rows):
+        sc[t, :len(r)] = r
+    bh = inputs.Batch(np.zeros(T, np.int64), np.array([len(r) for r in rows], np.int32),
+                      np.arange(T, dtype=np.int32), np.array([len(r) - 1 for r in rows], np.int32),
+                      np.zeros(T, np.int32))
+    db = B.DeviceBatch.from_host(bh, cuda_device, kv_rows=int(nmax))
+    s_dev = torch.from_numpy(sc).to(cuda_device)
+    idx = torch.full((T, k), -7, dtype=torch.int32, device=cuda_device)
+    ws = B.workspace(B.OP_TOPK, db, k=k, device=cuda_device)
+    B.dsa_topk(db, s_dev, ld, k, idx, ws)
+    assert B.read_device_status(ws) == 0
+    got = idx.cpu().numpy()
+    want = oracle.topk_select(sc, np.array([len(r) for r in rows]), k)
+    for t in range(T):
+        assert np.array_equal(got[t], want[t]), f"row {t} (n={len(rows[t])})"
+
+
+def test_topk_bit_exact_on_oracle_scores(cuda_device):
+    wl = WORKLOADS["tiny_prefill"]
+    ins = inputs.make_inputs(wl)
+    rows = []
+    for t in range(0, 1024, 7):
+        I, _ = H.indexer_ref_row(ins, t)
+        rows.append(I.astype(np.float32))
+    _topk_case(cuda_device, rows, wl.k)
+
+
+def test_topk_adversarial_rows(cuda_device):
+    rng = np.random.default_rng(11)
+    k = 2048
+    rows = [
+        rng.standard_normal(5000).astype(np.float32),
+        np.round(rng.standard_normal(6000), 1).astype(np.float32),          # heavy ties
+        np.zeros(4000, np.float32),                                           # all equal
+        np.where(rng.random(4500) < 0.5, -0.0, 0.0).astype(np.float32),      # signed zeros only
+        np.concatenate([np.full(100, 3.0), np.where(rng.random(4000) < 0.5, -0.0, 0.0)]).astype(np.float32),
+        rng.standard_normal(k - 1).astype(np.float32),
+        rng.standard_normal(k).astype(np.float32),
+        rng.standard_normal(k + 1).astype(np.float32),
+        (rng.standard_normal(9000) * 1e-30).astype(np.float32),             # subnormal-range values
+        np.concatenate([rng.standard_normal(3000), [np.inf, -np.inf, np.inf]]).astype(np.float32),
+        rng.integers(-3, 4, size=8192).astype(np.float32),
+        np.array([1.5], np.float32),
+    ]
+    _topk_case(cuda_device, rows, k)
+    _topk_case(cuda_device, rows[:5], 64)
+    _topk_case(cuda_device, [rng.standard_normal(n).astype(np.float32) for n in (300, 257, 256, 255)], 256)
+
+
+def test_topk_long_rows_from_l2(cuda_device):
+    rng = np.random.default_rng(12)
+    rows = [rng.standard_normal(40000).astype(np.float32),
+            np.round(rng.standard_normal(131072), 2).astype(np.float32),
+            rng.standard_normal(33000).astype(np.float32)]
+    _topk_case(cuda_device, rows, 2048)
+
+# ----------------------------------------------------------------------------- sparse MLA
+
+
+def _mla_ref_rows(ins, idx_host, rows, wl):
+    batch = ins["batch"]
+    refs, lses = [], []
+    for t in rows:
+        off, n = H.seq_slice(batch, t)
+        o, l = oracle.sparse_mla(oracle.bf16_decode(ins["q"][t:t + 1]), oracle.bf16_decode(ins["kv"][off:off + n]),
+                                 idx_host[t:t + 1].astype(np.int64), wl.sm_scale)
+        refs.append(o[0])
+        lses.append(l[0])
+    return np.stack(refs), np.stack(lses)
+
+
+def _run_mla(dev, wl, idx_host, T):
+    idx = torch.from_numpy(idx_host.astype(np.int32)).to(dev["q"].device)
+    out = torch.zeros((T, wl.heads, 512), dtype=torch.int16, device=idx.device)
+    lse = torch.zeros((T, wl.heads), dtype=torch.float32, device=idx.device)
+    ws = B.workspace(B.OP_SPARSE_MLA, dev["batch"], H=wl.heads, k=idx_host.shape[1], device=idx.device)
+    B.dsa_sparse_mla(dev["batch"], dev["q"], dev["kv"], idx, idx_host.shape[1], wl.heads, wl.sm_scale, out, lse, ws)
+    assert B.read_device_status(ws) == 0
+    return B.tensor_to_bits(out), lse.cpu().numpy()
+
+
+def _oracle_idx(ins, wl, rows=None):
+    batch = ins["batch"]
+    T = batch.num_q
+    idx = np.full((T, wl.k), -1, np.int32)
+    for t in (range(T) if rows is None else rows):
+        I, _ = H.indexer_ref_row(ins, t)
+        n = int(batch.q_pos[t]) + 1
+        idx[t] = oracle.topk_select(I[None, :n], np.array([n]), wl.k)[0]
+    return idx
+
+
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny_prefill"], MID_PREFILL, MID_DEC2, MID_DEC1], ids=lambda w: w.name)
+def test_sparse_mla_matches_oracle(cuda_device, wl):
+    ins = inputs.make_inputs(wl)
+    batch = ins["batch"]
+    T = batch.num_q
+    rows = list(range(T)) if T <= 64 else _sample_rows(T, wl.k)
+    idx = _oracle_idx(ins, wl, rows if T > 1100 else None)
+    dev = H.to_device(ins, cuda_device)
+    out_bits, lse = _run_mla(dev, wl, idx, T)
+    ref, ref_lse = _mla_ref_rows(ins, idx, rows, wl)
+    H.check_attention(out_bits[rows], ref, wl.name)
+    assert np.max(np.abs(lse[rows] - ref_lse)) <= H.LSE_ABS
+
+
+def test_sparse_mla_holes_unsorted_and_empty_rows(cuda_device):
+    wl = Workload("holes", 26, "decode", k=640, h_index=64, heads=128, batch=4, ctx_min=700, ctx_max=2000,
+                  q_per_seq=1)
+    ins = inputs.make_inputs(wl)
+    batch = ins["batch"]
+    T = batch.num_q
+    rng = np.random.default_rng(3)
+    idx = np.full((T, wl.k), -1, np.int32)
+    for t in range(T):
+        n = int(batch.q_pos[t]) + 1
+        sel = rng.choice(n, size=min(n, 500), replace=False).astype(np.int32)
+        slots = np.sort(rng.choice(wl.k, size=sel.size, replace=False))
+        idx[t, slots] = sel                     # unsorted, with -1 holes anywhere
+    idx[T - 1] = -1                             # a query with nothing selected
+    dev = H.to_device(ins, cuda_device)
+    out_bits, lse = _run_mla(dev, wl, idx, T)
+    ref, ref_lse = _mla_ref_rows(ins, idx, range(T - 1), wl)
+    H.check_attention(out_bits[:T - 1], ref, "holes")
+    assert np.max(np.abs(lse[:T - 1] - ref_lse)) <= H.LSE_ABS
+    assert np.all(oracle.bf16_decode(out_bits[T - 1]) == 0) and np.all(np.isneginf(lse[T - 1]))
+
+
+def test_sparse_mla_fewer_heads(cuda_device):
+    wl = Workload("h40", 27, "prefill", k=128, h_index=8, heads=40, seq_len=300)
+    ins = inputs.make_inputs(wl)
+    T = ins["batch"].num_q
+    idx = _oracle_idx(ins, wl)
+    out_bits, lse = _run_mla(H.to_device(ins, cuda_device), wl, idx, T)
+    ref, ref_lse = _mla_ref_rows(ins, idx, range(T), wl)
+    H.check_attention(out_bits, ref, "h40")
+
+# ----------------------------------------------------------------------------- end to end
+
+
+def _forward(dev, wl, batch_host):
+    T = batch_host.num_q
+    d = dev["q"].device
+    out = torch.zeros((T, wl.heads, 512), dtype=torch.int16, device=d)
+    lse = torch.zeros((T, wl.heads), dtype=torch.float32, device=d)
+    ws = B.workspace(B.OP_FORWARD, dev["batch"], H_I=wl.h_index, H=wl.heads, k=wl.k, device=d)
+    B.dsa_forward(dev["batch"], dev["q_idx"], dev["k_idx"], dev["w"], wl.h_index, dev["q"], dev["kv"], wl.heads,
+                  wl.k, wl.sm_scale, out, lse, ws)
+    assert B.read_device_status(ws) == 0
+    sp, ld, ip = B.forward_ws_views(dev["batch"], wl.h_index, wl.heads, wl.k, ws)
+    base = ws.data_ptr()
+    scores = ws[sp - base: sp - base + T * ld * 4].view(torch.float32).view(T, ld).cpu().numpy()
+    idx = ws[ip - base: ip - base + T * wl.k * 4].view(torch.int32).view(T, wl.k).cpu().numpy()
+    return B.tensor_to_bits(out), lse.cpu().numpy(), scores, idx
+
+
+def check_forward_rows(ins, wl, rows, out_bits, lse, scores, idx):
+    batch = ins["batch"]
+    mism = 0
+    for t in rows:
+        I, A = H.indexer_ref_row(ins, t)
+        n = int(batch.q_pos[t]) + 1
+        H.check_indexer_row(scores[t, :n], I, A, f"{wl.name} row {t}")
+        mism += H.check_selection(idx[t], I, n, wl.k, f"{wl.name} row {t}")
+    ref, ref_lse = _mla_ref_rows(ins, idx, rows, wl)       # the oracle's attention on the GPU's selection
+    H.check_attention(out_bits[rows], ref, wl.name)
+    assert np.max(np.abs(lse[rows] - ref_lse)) <= H.LSE_ABS
+    return mism
+
+
+@pytest.mark.parametrize("wl", [WORKLOADS["tiny_prefill"], MID_PREFILL, MID_DEC2], ids=lambda w: w.name)
+def test_forward_end_to_end(cuda_device, wl):
+    ins = inputs.make_inputs(wl)
+    batch = ins["batch"]
+    dev = H.to_device(ins, cuda_device)
+    out_bits, lse, scores, idx = _forward(dev, wl, batch)
+    T = batch.num_q
+    rows = list(range(T)) if T <= 64 else _sample_rows(T, wl.k)
+    check_forward_rows(ins, wl, rows, out_bits, lse, scores, idx)
+
+
+@pytest.mark.parametrize("name", ["prefill_8k", "decode_b64", "decode_128k_mtp2", "chunked_64k"])
+def test_forward_full_size_sampled(cuda_device, name):
+    """The five workloads at full size (the chunked one: its last chunk), through
+    dsa_forward as the benchmark runs it, checked on sampled rows."""
+    wl = WORKLOADS[name]
+    chunk = (wl.seq_len // wl.chunk - 1) if wl.kind == "chunked_prefill" else None
+    ins = inputs.make_inputs(wl, chunk_index=chunk)
+    batch = ins["batch"]
+    dev = H.to_device(ins, cuda_device)
+    out_bits, lse, scores, idx = _forward(dev, wl, batch)
+    T = batch.num_q
+    rows = _sample_rows(T, wl.k) if T > 64 else list(range(0, T, max(1, T // 16)))
+    check_forward_rows(ins, wl, rows[:20], out_bits, lse, scores, idx)
+
+# ----------------------------------------------------------------------------- device status
+
+
+def test_device_status_flags_bad_queries_and_indices(cuda_device):
+    wl = Workload("bad", 28, "decode", k=128, h_index=64, heads=128, batch=2, ctx_min=200, ctx_max=300,
+                  q_per_seq=1)
+    ins = inputs.make_inputs(wl)
+    bh = ins["batch"]
+    bad = inputs.Batch(bh.kv_offset, bh.kv_len, bh.q_seq, bh.q_pos.copy(), bh.q_row)
+    bad.q_pos[1] = bh.kv_len[1] + 5                       # beyond its sequence
+    dev = H.to_device({**ins, "batch": bad}, cuda_device)
+    T = 2
+    ld = (int(bh.kv_len.max()) + 3) // 4 * 4
+    scores = torch.zeros((T, ld), device=cuda_device)
+    ws = B.workspace(B.OP_INDEXER, dev["batch"], ld=ld, device=cuda_device)
+    B.dsa_indexer_scores(dev["batch"], dev["q_idx"], dev["k_idx"], dev["w"], 64, scores, ld, ws)
+    assert B.read_device_status(ws) & B.DEV_BAD_QUERY
+    idx = torch.full((T, wl.k), -1, dtype=torch.int32, device=cuda_device)
+    ws2 = B.workspace(B.OP_TOPK, dev["batch"], k=wl.k, device=cuda_device)
+    B.dsa_topk(dev["batch"], scores, ld, wl.k, idx, ws2)
+    assert B.read_device_status(ws2) & B.DEV_BAD_QUERY
+    assert (idx[1] == -1).all()
+    good = H.to_device(ins, cuda_device)
+    idx_h = np.full((T, wl.k), -1, np.int32)
+    idx_h[:, 0] = 0
+    idx_h[0, 1] = int(bh.kv_len[0]) + 3                   # out of range
+    out_bits, _ = None, None
+    i_dev = torch.from_numpy(idx_h).to(cuda_device)
+    out = torch.zeros((T, 128, 512), dtype=torch.int16, device=cuda_device)
+    ws3 = B.workspace(B.OP_SPARSE_MLA, good["batch"], H=128, k=wl.k, device=cuda_device)
+    B.dsa_sparse_mla(good["batch"], good["q"], good["kv"], i_dev, wl.k, 128, wl.sm_scale, out, None, ws3)
+    assert B.read_device_status(ws3) & B.DEV_BAD_INDEX

@@ -1,0 +1,95 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every declared entry
+point, reports its version and status names, sizes workspaces, and rejects
+bad arguments on the host before touching the GPU."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from sparse_attention_weight_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^[\w \*]+?\b(dsa_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_attention_weight_b200 import build
+    build.build()
+    return B.lib()
+
+
+def test_library_exports_every_declared_function(lib):
+    names = _declared_functions()
+    assert set(B.EXPORTS) <= set(names) and len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dsa_abi_version() == 1
+    for code, name in B.STATUS_NAMES.items():
+        assert lib.dsa_status_string(code).decode() == name
+
+
+def _fake_batch(T=16, Bn=2, max_len=3000, kv_rows=6000):
+    # fake, aligned device addresses: never dereferenced by the failing calls below
+    return B.DsaBatch(Bn, T, max_len, 0, kv_rows, 0x10000, 0x20000, 0x30000, 0x40000)
+
+
+def test_workspace_sizes(lib):
+    b = _fake_batch()
+    sz = lambda op, **kw: lib.dsa_workspace_size(op, ctypes.byref(b), kw.get("hi", 64), kw.get("h", 128),
+                                                 kw.get("k", 2048), kw.get("ld", 0))
+    assert sz(B.OP_TOPK) >= 256
+    assert sz(B.OP_INDEXER) >= 256 + (6 * 16 + 2) * 4
+    fwd = sz(B.OP_FORWARD)
+    assert fwd >= 16 * 3000 * 4 + 16 * 2048 * 4
+    assert sz(B.OP_FORWARD, h=7) == 0 and sz(9) == 0
+    assert lib.dsa_workspace_size(0, None, 64, 128, 2048, 0) == 0
+
+
+def test_host_argument_checks(lib):
+    b = _fake_batch()
+    ws = 0x50000
+    p = 0x60000
+    big = 1 << 40
+    # null batch / workspace
+    assert lib.dsa_topk(None, p, 3000, 2048, p, ws, big, None) == 1
+    assert lib.dsa_topk(ctypes.byref(b), p, 3000, 2048, p, None, big, None) == 1
+    # unsupported shapes
+    assert lib.dsa_indexer_scores(ctypes.byref(b), p, p, p, 12, p, 3000, ws, big, None) == 2
+    assert lib.dsa_indexer_scores(ctypes.byref(b), p, p, p, 64, p, 2999, ws, big, None) == 2   # ld % 4
+    assert lib.dsa_indexer_scores(ctypes.byref(b), p, p, p, 64, p, 2000, ws, big, None) == 2   # ld < max_kv_len
+    assert lib.dsa_topk(ctypes.byref(b), p, 3000, 4096, p, ws, big, None) == 2
+    assert lib.dsa_topk(ctypes.byref(b), p, 3000, 0, p, ws, big, None) == 2
+    assert lib.dsa_sparse_mla(ctypes.byref(b), p, p, p, 2048, 12, 0.1, p, None, ws, big, None) == 2
+    assert lib.dsa_sparse_mla(ctypes.byref(b), p + 2, p, p, 2048, 128, 0.1, p, None, ws, big, None) == 2  # alignment
+    # workspace too small
+    assert lib.dsa_forward(ctypes.byref(b), p, p, p, 64, p, p, 128, 2048, 0.1, p, None, ws, 1024, None) == 3
+    # bad batch fields
+    bad = B.DsaBatch(0, 16, 3000, 0, 6000, 1, 1, 1, 1)
+    assert lib.dsa_topk(ctypes.byref(bad), p, 3000, 2048, p, ws, big, None) == 1
+    nulls = B.DsaBatch(2, 16, 3000, 0, 6000, 0, 0, 0, 0)
+    assert lib.dsa_topk(ctypes.byref(nulls), p, 3000, 2048, p, ws, big, None) == 1
+
+
+def test_read_device_status_rejects_null(lib):
+    flags = ctypes.c_uint32()
+    assert lib.dsa_read_device_status(None, ctypes.byref(flags), None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        B.lib()
