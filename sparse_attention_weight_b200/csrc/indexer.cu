@@ -12,8 +12,9 @@
 // Keys sit in TMEM lanes, so the per-head ReLU, weighting and head sum of the
 // epilogue run along one thread's own columns with no cross-lane reduction,
 // and each warp stores 32 consecutive scores of a row (coalesced).
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..5 epilogue.  The grid is persistent (one CTA per SM); each
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..9 epilogue (two warps per TMEM lane quadrant, splitting the
+// group's tokens).  The grid is persistent (one CTA per SM); each
 // CTA takes a contiguous range of work items so the resident query tile is
 // reused across the key tiles of its group.
 #include <cstdio>
@@ -25,7 +26,8 @@ namespace dsa {
 
 namespace {
 
-constexpr int kIdxThreads = 192;
+constexpr int kIdxThreads = 320;
+constexpr int kEpiWarps = 8;
 constexpr int kKeyTile = 128;        // keys per item (MMA M)
 constexpr int kStages = 6;           // key-tile ring depth
 constexpr int kTileBytes = kKeyTile * DSA_D_INDEX;   // 16 KB
@@ -34,8 +36,8 @@ constexpr int kQBytes = 256 * DSA_D_INDEX;           // 32 KB (N <= 256)
 struct __align__(8) IdxSmem {
   uint8_t q[kQBytes];                  // 1024-aligned (offset 0)
   uint8_t k[kStages][kTileBytes];      // 1024-aligned
-  float w[4][256];                     // per epilogue warp: head weights of the group
-  int32_t n_vis[4][256];               // per epilogue warp: visible keys per token
+  float w[kEpiWarps][256];             // per epilogue warp: head weights of the group
+  int32_t n_vis[kEpiWarps][256];       // per epilogue warp: visible keys per token
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t q_full, q_empty;
   uint64_t acc_full[2], acc_empty[2];
@@ -75,7 +77,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int s = 0; s < kStages; ++s) { mbar_init(&S.k_full[s], 1); mbar_init(&S.k_empty[s], 1); }
     mbar_init(&S.q_full, 1);
     mbar_init(&S.q_empty, 1);
-    for (int a = 0; a < 2; ++a) { mbar_init(&S.acc_full[a], 1); mbar_init(&S.acc_empty[a], 128); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&S.acc_full[a], 1); mbar_init(&S.acc_empty[a], 32 * kEpiWarps); }
     mbar_init(&S.done, 1);
     S.abort_flag = 0;
     fence_mbar_init();
@@ -93,11 +95,12 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       // ------------------------------------------------------------ producer
       if (lane == 0) {
         int g = find_group(p.item_off, ngroups, i0);
+        int g_lo = p.item_off[g], g_hi = p.item_off[g + 1];
         int prev_g = -1, issued = 0, q_loads = 0;
         uint32_t qe_par = 0;
         for (int i = i0; i < i1; ++i) {
-          while (p.item_off[g + 1] <= i) ++g;
-          const int kt = i - p.item_off[g];
+          while (g_hi <= i) { ++g; g_lo = g_hi; g_hi = p.item_off[g + 1]; }
+          const int kt = i - g_lo;
           if (g != prev_g) {
             if (prev_g >= 0) {
               if (!mbar_wait(&S.q_empty, qe_par, p.status, abort_flag)) break;
@@ -126,10 +129,11 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (lane == 0) {
         const uint32_t idesc = instr_desc(0, 0, false, false, kKeyTile, N);
         int g = find_group(p.item_off, ngroups, i0);
+        int g_hi = p.item_off[g + 1];
         int prev_g = -1;
         uint32_t qf_par = 0;
         for (int i = i0; i < i1; ++i) {
-          while (p.item_off[g + 1] <= i) ++g;
+          while (g_hi <= i) { ++g; g_hi = p.item_off[g + 1]; }
           if (g != prev_g) {
             if (!mbar_wait(&S.q_full, qf_par, p.status, abort_flag)) break;
             qf_par ^= 1;
@@ -152,7 +156,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           umma_commit(&S.k_empty[st]);
           umma_commit(&S.acc_full[a]);
-          const bool last_of_group = (i + 1 == i1) || (p.item_off[g + 1] <= i + 1);
+          const bool last_of_group = (i + 1 == i1) || (g_hi <= i + 1);
           if (last_of_group) umma_commit(&S.q_empty);
         }
         umma_commit(&S.done);
@@ -161,15 +165,18 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else {
       // ------------------------------------------------------------ epilogue
       // Warp-uniform control flow: lane 0 waits on barriers, the warp follows.
+      const int ew = warp - 2;                    // 0..7
       const int quad = warp & 3;                  // TMEM lane quadrant of this warp
+      const int tsub = ew >> 2;                   // token parity handled by this warp
       const int row = quad * 32 + lane;           // key within the tile
-      float* sw = S.w[warp - 2];
-      int32_t* snv = S.n_vis[warp - 2];
+      float* sw = S.w[ew];
+      int32_t* snv = S.n_vis[ew];
       int g = find_group(p.item_off, ngroups, i0);
+      int g_lo = p.item_off[g], g_hi = p.item_off[g + 1];
       int prev_g = -1, cnt = 0, q0 = 0;
       for (int i = i0; i < i1; ++i) {
-        while (p.item_off[g + 1] <= i) ++g;
-        const int kt = i - p.item_off[g];
+        while (g_hi <= i) { ++g; g_lo = g_hi; g_hi = p.item_off[g + 1]; }
+        const int kt = i - g_lo;
         if (g != prev_g) {
           __syncwarp();
           q0 = p.group_q0[g];
@@ -189,29 +196,28 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int s = kt * kKeyTile + row;
         const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + a * 256;
         if constexpr (HI >= 32) {
-          for (int tok = 0; tok < cnt; ++tok) {
-            float acc = 0.f;
+          for (int tok = tsub; tok < cnt; tok += 2) {
+            uint32_t v[HI];
 #pragma unroll
-            for (int c = 0; c < HI / 32; ++c) {
-              uint32_t v[32];
-              tmem_ld32(tbase + tok * HI + c * 32, v);
-              tmem_ld_wait();
-              const float* wr = &sw[tok * HI + c * 32];
+            for (int c = 0; c < HI / 32; ++c)
+              tmem_ld32(tbase + tok * HI + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+            tmem_ld_wait();
+            const float* wr = &sw[tok * HI];
+            float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                const float4 w4 = *reinterpret_cast<const float4*>(wr + j);
-                acc = fmaf(w4.x, fmaxf(__uint_as_float(v[j + 0]), 0.f), acc);
-                acc = fmaf(w4.y, fmaxf(__uint_as_float(v[j + 1]), 0.f), acc);
-                acc = fmaf(w4.z, fmaxf(__uint_as_float(v[j + 2]), 0.f), acc);
-                acc = fmaf(w4.w, fmaxf(__uint_as_float(v[j + 3]), 0.f), acc);
-              }
+            for (int j = 0; j < HI; j += 4) {
+              const float4 w4 = *reinterpret_cast<const float4*>(wr + j);
+              acc0 = fmaf(w4.x, fmaxf(__uint_as_float(v[j + 0]), 0.f), acc0);
+              acc1 = fmaf(w4.y, fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
+              acc0 = fmaf(w4.z, fmaxf(__uint_as_float(v[j + 2]), 0.f), acc0);
+              acc1 = fmaf(w4.w, fmaxf(__uint_as_float(v[j + 3]), 0.f), acc1);
             }
-            if (s < snv[tok]) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = acc;
+            if (s < snv[tok]) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = acc0 + acc1;
           }
         } else {
           constexpr int TPC = 32 / HI;             // tokens per 32-column chunk
           const int nchunks = (cnt * HI + 31) / 32;
-          for (int c = 0; c < nchunks; ++c) {
+          for (int c = tsub; c < nchunks; c += 2) {
             uint32_t v[32];
             tmem_ld32(tbase + c * 32, v);
             tmem_ld_wait();

@@ -26,7 +26,11 @@
 //
 // Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-5 gather of the
 // S operand rows, 6-7 gather of the V operand rows, 8 TMEM owner and (in the
-// even CTA) MMA issuer.
+// even CTA) MMA issuer, 9 relay.  Gather threads never wait for their own
+// copies: each arrives on a local stage barrier through cp.async.mbarrier.arrive
+// (hardware-tracked completion), and a relay lane that has no copies in flight
+// forwards the completed stage to the even CTA's barrier, which the MMA issuer
+// waits on.
 #include <cuda_bf16.h>
 
 #include "dsa_common.cuh"
@@ -36,13 +40,12 @@ namespace dsa {
 
 namespace {
 
-constexpr int kMlaThreads = 288;
+constexpr int kMlaThreads = 320;
 constexpr int kBlk = 128;             // selected rows per block (pair)
 constexpr int kHalf = 64;             // rows per CTA for the S operand; heads per CTA
 constexpr int kDChunks = DSA_D_QK / 64;   // 9 chunks of 64 dims
 constexpr int kSStages = 8;           // S-operand ring (8 KB slots)
 constexpr int kVStages = 6;           // V-operand ring (8 KB slots)
-constexpr int kLag = 3;               // cp.async groups kept in flight per producer thread
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr uint32_t kSCol = 0;         // TMEM columns [0,128): two S buffers of 64
 constexpr uint32_t kOCol = 128;       // TMEM columns [128,384): O (2 x 128)
@@ -55,8 +58,8 @@ struct __align__(1024) MlaSmem {
   float xmax[2][128];
   float lsum[128];
   uint64_t q_full, q_ready;
-  uint64_t s_full[kSStages], s_empty[kSStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[kSStages], s_empty[kSStages], s_loaded[kSStages];
+  uint64_t v_full[kVStages], v_empty[kVStages], v_loaded[kVStages];
   uint64_t s_ready[2], s_free[2];
   uint64_t p_full, p_empty;
   uint64_t mx_bar[2], l_bar;
@@ -78,9 +81,11 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// Arrive on `bar` once every cp.async issued so far by this thread has completed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
@@ -129,8 +134,12 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
   if (threadIdx.x == 0) {
     mbar_init(&S.q_full, 1);
     mbar_init(&S.q_ready, 2);
-    for (int i = 0; i < kSStages; ++i) { mbar_init(&S.s_full[i], 4); mbar_init(&S.s_empty[i], 1); }
-    for (int i = 0; i < kVStages; ++i) { mbar_init(&S.v_full[i], 4); mbar_init(&S.v_empty[i], 1); }
+    for (int i = 0; i < kSStages; ++i) {
+      mbar_init(&S.s_full[i], 2); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], 64);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&S.v_full[i], 2); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], 64);
+    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 8); mbar_init(&S.mx_bar[i], 128);
     }
@@ -331,57 +340,57 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         if (mbar_wait(&S.q_full, 0, p.status, ab)) mbar_arrive_cluster(&S.q_ready, 0);
       }
       const int nchunks = nblk * kDChunks;
-      for (int n = 0; n < nchunks + kLag; ++n) {
-        if (n < nchunks) {
-          const int j = n / kDChunks, dc = n % kDChunks, st = n % kSStages;
-          if (!warp_wait(&S.s_empty[st], ((n / kSStages) & 1) ^ 1, p.status, ab, false)) break;
-          const uint32_t dst0 = smem_u32(S.s_ring[st]);
+      for (int n = 0; n < nchunks; ++n) {
+        const int j = n / kDChunks, dc = n % kDChunks, st = n % kSStages;
+        if (!warp_wait(&S.s_empty[st], ((n / kSStages) & 1) ^ 1, p.status, ab, false)) break;
+        const uint32_t dst0 = smem_u32(S.s_ring[st]);
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int r = it * 8 + (pt >> 3);                  // row within this CTA's 64
-            const int64_t g = sel_row(p, idx_row, (blk0 + j) * kBlk + static_cast<int>(rank) * kHalf + r, base, len);
-            const uint16_t* src = p.kv + (g < 0 ? 0 : g) * DSA_D_QK + dc * 64 + c16 * 8;
-            cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4), src, g < 0 ? 0u : 16u);
-          }
+        for (int it = 0; it < 8; ++it) {
+          const int r = it * 8 + (pt >> 3);                    // row within this CTA's 64
+          const int64_t g = sel_row(p, idx_row, (blk0 + j) * kBlk + static_cast<int>(rank) * kHalf + r, base, len);
+          const uint16_t* src = p.kv + (g < 0 ? 0 : g) * DSA_D_QK + dc * 64 + c16 * 8;
+          cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4), src, g < 0 ? 0u : 16u);
         }
-        cp_async_commit();
-        if (n >= kLag) {
-          cp_async_wait<kLag>();
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(&S.s_full[(n - kLag) % kSStages], 0);
-        }
+        cp_async_arrive_noinc(&S.s_loaded[st]);
       }
-      cp_async_wait<0>();
+      cp_async_wait_all();
     } else if (warp < 8) {
       // ================================================================ V-operand gather
       const int pt = threadIdx.x - 192;                      // 0..63
       const int c16 = pt & 7;
       const int nchunks = nblk * (kBlk / 16);
-      for (int n = 0; n < nchunks + kLag; ++n) {
-        if (n < nchunks) {
-          const int j = n / (kBlk / 16), kk = n % (kBlk / 16), st = n % kVStages;
-          if (!warp_wait(&S.v_empty[st], ((n / kVStages) & 1) ^ 1, p.status, ab, false)) break;
-          const uint32_t dst0 = smem_u32(S.v_ring[st]);
+      for (int n = 0; n < nchunks; ++n) {
+        const int j = n / (kBlk / 16), kk = n % (kBlk / 16), st = n % kVStages;
+        if (!warp_wait(&S.v_empty[st], ((n / kVStages) & 1) ^ 1, p.status, ab, false)) break;
+        const uint32_t dst0 = smem_u32(S.v_ring[st]);
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int pi = it * 8 + (pt >> 3);                 // (row, group) pair 0..63
-            const int r = pi & 15, grp = pi >> 4;
-            const int d0 = (grp >> 1) * 256 + static_cast<int>(rank) * 128 + (grp & 1) * 64;
-            const int64_t g = sel_row(p, idx_row, (blk0 + j) * kBlk + kk * 16 + r, base, len);
-            const uint16_t* src = p.kv + (g < 0 ? 0 : g) * DSA_D_QK + d0 + c16 * 8;
-            cp_async16(dst0 + grp * 2048 + r * 128 + ((c16 ^ (r & 7)) << 4), src, g < 0 ? 0u : 16u);
-          }
+        for (int it = 0; it < 8; ++it) {
+          const int pi = it * 8 + (pt >> 3);                   // (row, group) pair 0..63
+          const int r = pi & 15, grp = pi >> 4;
+          const int d0 = (grp >> 1) * 256 + static_cast<int>(rank) * 128 + (grp & 1) * 64;
+          const int64_t g = sel_row(p, idx_row, (blk0 + j) * kBlk + kk * 16 + r, base, len);
+          const uint16_t* src = p.kv + (g < 0 ? 0 : g) * DSA_D_QK + d0 + c16 * 8;
+          cp_async16(dst0 + grp * 2048 + r * 128 + ((c16 ^ (r & 7)) << 4), src, g < 0 ? 0u : 16u);
         }
-        cp_async_commit();
-        if (n >= kLag) {
-          cp_async_wait<kLag>();
+        cp_async_arrive_noinc(&S.v_loaded[st]);
+      }
+      cp_async_wait_all();
+    } else if (warp == 9) {
+      // ================================================================ relay
+      // lane 0: S stages, lane 1: V stages.  Local completion -> the even CTA.
+      if (lane < 2) {
+        const bool is_s = lane == 0;
+        const int nchunks = is_s ? nblk * kDChunks : nblk * (kBlk / 16);
+        const int stages = is_s ? kSStages : kVStages;
+        uint64_t* loaded = is_s ? S.s_loaded : S.v_loaded;
+        uint64_t* full = is_s ? S.s_full : S.v_full;
+        for (int n = 0; n < nchunks; ++n) {
+          const int st = n % stages;
+          if (!mbar_wait(&loaded[st], (n / stages) & 1, p.status, ab)) break;
           fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(&S.v_full[(n - kLag) % kVStages], 0);
+          mbar_arrive_cluster(&full[st], 0);
         }
       }
-      cp_async_wait<0>();
     } else if (rank == 0 && lane == 0) {
       // ================================================================ MMA issuer (even CTA)
       const uint32_t id_s = instr_desc(1, 1, false, false, 128, kBlk);   // bf16 x bf16, M=128 pair, N=128

@@ -11,7 +11,8 @@ from sparse_attention_weight_b200 import inputs
 
 # Tolerances (stated per check):
 #   indexer scores: |I_gpu - I_ref| <= 1e-4 * max(|I_ref|, A_ref), A_ref = sum_j |w_j| ReLU(dot_j)
-#   attention output (bf16 I/O) vs the fp64 oracle: max-abs <= 1e-2, mean-abs <= 1e-3
+#   attention output (bf16 I/O) vs the fp64 oracle: max-abs <= 1e-2 beyond the bf16 rounding of
+#   the output (2^-8 |ref|), mean-abs <= 1e-3
 #   lse: abs <= 2e-3 (fp32 softmax statistics; a derived bound)
 IDX_RTOL = 1e-4
 OUT_MAX_ABS = 1e-2
@@ -59,10 +60,19 @@ def check_indexer_row(got: np.ndarray, I: np.ndarray, A: np.ndarray, what: str):
 
 
 def check_attention(out_bits: np.ndarray, ref: np.ndarray, what: str):
+    """Output of a bf16-I/O attention against the fp64 oracle.
+
+    max-abs: |out - ref| <= 1e-2 + 2^-8 |ref|.  The second term is the rounding of
+    the result into the bf16 output format (half an ulp is at most 2^-8 of the
+    value; it alone reaches 0.0156 for |x| in [4, 8)), which no bf16 output can
+    avoid; 1e-2 bounds the computational error on top of it.
+    mean-abs: mean |out - ref| <= 1e-3.
+    """
     got = oracle.bf16_decode(out_bits)
     err = np.abs(got - ref)
-    assert err.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS, (
-        f"{what}: max-abs {err.max():.3e} mean-abs {err.mean():.3e}")
+    excess = err - 2.0 ** -8 * np.abs(ref)
+    assert excess.max() <= OUT_MAX_ABS and err.mean() <= OUT_MEAN_ABS, (
+        f"{what}: max-abs {err.max():.3e} (beyond bf16 rounding {excess.max():.3e}) mean-abs {err.mean():.3e}")
     return float(err.max()), float(err.mean())
 
 

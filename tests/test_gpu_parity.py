@@ -45,7 +45,7 @@ def _sample_rows(T, k, extra=()):
 def _run_indexer(dev, wl, batch_host):
     T = batch_host.num_q
     ld = (batch_host.max_kv_len + 3) // 4 * 4
-    scores = torch.full((T, ld), float("nan"), device=dev)
+    scores = torch.full((T, ld), float("nan"), device=dev["q"].device)
     ws = B.workspace(B.OP_INDEXER, dev["batch"], H_I=wl.h_index, ld=ld, device=scores.device)
     B.dsa_indexer_scores(dev["batch"], dev["q_idx"], dev["k_idx"], dev["w"], wl.h_index, scores, ld, ws)
     assert B.read_device_status(ws) == 0
