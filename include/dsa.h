@@ -62,6 +62,7 @@ typedef enum dsa_status {
 #define DSA_DEV_BAD_QUERY 1u      /* q_seq out of [0,B) or q_pos out of [0, kv_len) */
 #define DSA_DEV_BAD_INDEX 2u      /* a selected index >= kv_len of its sequence */
 #define DSA_DEV_TIMEOUT 4u        /* a bounded in-kernel wait expired; results invalid */
+#define DSA_DEV_INTERNAL 8u       /* a kernel precondition failed (e.g. shared-memory alignment); results invalid */
 
 typedef struct dsa_batch {
   int32_t num_seqs;        /* B >= 1 */

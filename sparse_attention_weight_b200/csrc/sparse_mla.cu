@@ -44,19 +44,20 @@ constexpr int kMlaThreads = 320;
 constexpr int kBlk = 128;             // selected rows per block (pair)
 constexpr int kHalf = 64;             // rows per CTA for the S operand; heads per CTA
 constexpr int kDChunks = DSA_D_QK / 64;   // 9 chunks of 64 dims
-constexpr int kSStages = 8;           // S-operand ring (8 KB slots)
-constexpr int kVStages = 6;           // V-operand ring (8 KB slots)
+constexpr int kSStages = 9;           // S-operand ring (8 KB slots): one full block
+constexpr int kVStages = 8;           // V-operand ring (8 KB slots): one full block
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr uint32_t kSCol = 0;         // TMEM columns [0,128): two S buffers of 64
 constexpr uint32_t kOCol = 128;       // TMEM columns [128,384): O (2 x 128)
 
-struct __align__(1024) MlaSmem {
+struct MlaSmem {
   uint8_t q[kDChunks][kHalf * 128];          // 72 KB  Q of this CTA's heads (K-major SW128)
   uint8_t s_ring[kSStages][kHalf * 128];     // 64 KB  S operand chunks: 64 rows x 64 dims
   uint8_t v_ring[kVStages][4][16 * 128];     // 48 KB  V operand chunks: 16 rows x 4 dim groups
   uint8_t p[2][kHalf * 128];                 // 16 KB  P: 64 heads x 128 rows (two K chunks)
   float xmax[2][128];
   float lsum[128];
+  uint32_t valid[2048 / 32];                 // bit e: entry e of the index row is a usable row
   uint64_t q_full, q_ready;
   uint64_t s_full[kSStages], s_empty[kSStages], s_loaded[kSStages];
   uint64_t v_full[kVStages], v_empty[kVStages], v_loaded[kVStages];
@@ -101,21 +102,22 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// Global row of selected entry `pos` of query t, or -1 when unused/invalid.
-__device__ __forceinline__ int64_t sel_row(const MlaParams& p, const int32_t* idx_row, int pos, int64_t base,
-                                           int len) {
-  if (pos >= p.k) return -1;
-  const int i = __ldg(idx_row + pos);
-  if (i < 0) return -1;
-  if (i >= len) { set_status(p.status, DSA_DEV_BAD_INDEX); return -1; }
-  return base + i;
+// Local row indices of block `blk` of query t's index row: r[s] = entry
+// blk*128 + 32*s + lane, or -1 when unused or out of range.
+__device__ __forceinline__ void block_rows(const MlaParams& p, const int32_t* idx_row, int blk, int len, int lane,
+                                           int (&r)[4]) {
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const int pos = blk * kBlk + 32 * s + lane;
+    const int v = pos < p.k ? __ldg(idx_row + pos) : -1;
+    r[s] = (v >= 0 && v < len) ? v : -1;
+  }
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
 sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  MlaSmem& S = *reinterpret_cast<MlaSmem*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  MlaSmem& S = *reinterpret_cast<MlaSmem*>(smem_raw);   // 1024-aligned: checked below
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const int cid = blockIdx.x >> 1;
@@ -148,15 +150,26 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
     mbar_init(&S.l_bar, 128);
     mbar_init(&S.done, 1);
     S.abort_flag = 0;
+    if (smem_u32(smem_raw) & 1023u) {           // the swizzled tiles need 1024-byte alignment
+      set_status(p.status, DSA_DEV_INTERNAL);
+      S.abort_flag = 1;
+    }
     fence_mbar_init();
     if (!rows_ok) set_status(p.status, DSA_DEV_BAD_QUERY);
   }
   // blocks of 128 entries covering the used part of the index row, split evenly
   if (warp == 4) {
     int last = -1;
-    if (rows_ok) {
-      for (int i = lane; i < p.k; i += 32)
-        if (__ldg(idx_row + i) >= 0) last = i;
+    for (int b = 0; b < 2048 / 32; ++b) {
+      const int i = b * 32 + lane;
+      int v = -1;
+      if (rows_ok && i < p.k) {
+        v = __ldg(idx_row + i);
+        if (v >= len) { set_status(p.status, DSA_DEV_BAD_INDEX); v = -1; }
+      }
+      if (v >= 0) last = i;
+      const uint32_t m = __ballot_sync(0xffffffffu, v >= 0);
+      if (lane == 0) S.valid[b] = m;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
@@ -174,7 +187,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
-  const int nblk = S.nblk;
+  const int nblk = S.abort_flag ? 0 : S.nblk;
   const int blk0 = S.blk0;
 
   const int H = p.H;
@@ -192,15 +205,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         const int sb = j & 1;
         const uint32_t sph = (j >> 1) & 1;
         // validity of this warp's 64 columns
-        const int pos0 = (blk0 + j) * kBlk + half * 64;
-        uint32_t vm0, vm1;
-        {
-          const int pa = pos0 + lane, pb = pos0 + 32 + lane;
-          const bool va = pa < p.k && __ldg(idx_row + pa) >= 0 && __ldg(idx_row + pa) < len;
-          const bool vb = pb < p.k && __ldg(idx_row + pb) >= 0 && __ldg(idx_row + pb) < len;
-          vm0 = __ballot_sync(0xffffffffu, va);
-          vm1 = __ballot_sync(0xffffffffu, vb);
-        }
+        const int pos0 = (blk0 + j) * kBlk + half * 64;      // multiple of 64
+        const uint32_t vm0 = pos0 < 2048 ? S.valid[pos0 >> 5] : 0u;
+        const uint32_t vm1 = pos0 + 32 < 2048 ? S.valid[(pos0 >> 5) + 1] : 0u;
         if (!warp_wait(&S.s_ready[sb], sph, p.status, ab, false)) break;
         tc_fence_after();
         uint32_t sr[64];
@@ -332,53 +339,79 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       // ================================================================ S-operand gather
       const int pt = threadIdx.x - 128;                      // 0..63
       const int c16 = pt & 7;
-      if (threadIdx.x == 128) {
-        // this CTA's 64 heads of Q: 9 TMA boxes of 64 dims x 64 rows
-        mbar_arrive_expect_tx(&S.q_full, kDChunks * kHalf * 128);
-        for (int dc = 0; dc < kDChunks; ++dc)
-          tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
-        if (mbar_wait(&S.q_full, 0, p.status, ab)) mbar_arrive_cluster(&S.q_ready, 0);
-      }
-      const int nchunks = nblk * kDChunks;
-      for (int n = 0; n < nchunks; ++n) {
-        const int j = n / kDChunks, dc = n % kDChunks, st = n % kSStages;
-        if (!warp_wait(&S.s_empty[st], ((n / kSStages) & 1) ^ 1, p.status, ab, false)) break;
-        const uint32_t dst0 = smem_u32(S.s_ring[st]);
+      // index entries of block j: lane holds entries 32*s + lane (s = 0..3), prefetched a block ahead
+      int cur[4], nxt[4];
+      block_rows(p, idx_row, blk0, len, lane, cur);
+      if (nblk > 1) block_rows(p, idx_row, blk0 + 1, len, lane, nxt);
+      bool ok = true;
+      int n = 0;
+      for (int j = 0; j < nblk && ok; ++j) {
+        if (j > 0) {
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int r = it * 8 + (pt >> 3);                    // row within this CTA's 64
-          const int64_t g = sel_row(p, idx_row, (blk0 + j) * kBlk + static_cast<int>(rank) * kHalf + r, base, len);
-          const uint16_t* src = p.kv + (g < 0 ? 0 : g) * DSA_D_QK + dc * 64 + c16 * 8;
-          cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4), src, g < 0 ? 0u : 16u);
+          for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
+          if (j + 1 < nblk) block_rows(p, idx_row, blk0 + j + 1, len, lane, nxt);
         }
-        cp_async_arrive_noinc(&S.s_loaded[st]);
+        for (int dc = 0; dc < kDChunks; ++dc, ++n) {
+          const int st = n % kSStages;
+          if (!warp_wait(&S.s_empty[st], ((n / kSStages) & 1) ^ 1, p.status, ab, false)) { ok = false; break; }
+          const uint32_t dst0 = smem_u32(S.s_ring[st]);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int r = it * 8 + (pt >> 3);                  // row within this CTA's 64
+            // entry rank*64 + r of the block: register slot rank*2 + it/4, lane (it%4)*8 + pt/8
+            const int mine = rank ? cur[2 + (it >> 2)] : cur[it >> 2];
+            const int v = __shfl_sync(0xffffffffu, mine, (it & 3) * 8 + (pt >> 3));
+            const uint16_t* src = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + dc * 64 + c16 * 8;
+            cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4), src, v < 0 ? 0u : 16u);
+          }
+          cp_async_arrive_noinc(&S.s_loaded[st]);
+        }
       }
       cp_async_wait_all();
     } else if (warp < 8) {
       // ================================================================ V-operand gather
       const int pt = threadIdx.x - 192;                      // 0..63
       const int c16 = pt & 7;
-      const int nchunks = nblk * (kBlk / 16);
-      for (int n = 0; n < nchunks; ++n) {
-        const int j = n / (kBlk / 16), kk = n % (kBlk / 16), st = n % kVStages;
-        if (!warp_wait(&S.v_empty[st], ((n / kVStages) & 1) ^ 1, p.status, ab, false)) break;
-        const uint32_t dst0 = smem_u32(S.v_ring[st]);
+      int cur[4], nxt[4];
+      block_rows(p, idx_row, blk0, len, lane, cur);
+      if (nblk > 1) block_rows(p, idx_row, blk0 + 1, len, lane, nxt);
+      bool ok = true;
+      int n = 0;
+      for (int j = 0; j < nblk && ok; ++j) {
+        if (j > 0) {
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int pi = it * 8 + (pt >> 3);                   // (row, group) pair 0..63
-          const int r = pi & 15, grp = pi >> 4;
-          const int d0 = (grp >> 1) * 256 + static_cast<int>(rank) * 128 + (grp & 1) * 64;
-          const int64_t g = sel_row(p, idx_row, (blk0 + j) * kBlk + kk * 16 + r, base, len);
-          const uint16_t* src = p.kv + (g < 0 ? 0 : g) * DSA_D_QK + d0 + c16 * 8;
-          cp_async16(dst0 + grp * 2048 + r * 128 + ((c16 ^ (r & 7)) << 4), src, g < 0 ? 0u : 16u);
+          for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
+          if (j + 1 < nblk) block_rows(p, idx_row, blk0 + j + 1, len, lane, nxt);
         }
-        cp_async_arrive_noinc(&S.v_loaded[st]);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk, ++n) {
+          const int st = n % kVStages;
+          if (!warp_wait(&S.v_empty[st], ((n / kVStages) & 1) ^ 1, p.status, ab, false)) { ok = false; break; }
+          const uint32_t dst0 = smem_u32(S.v_ring[st]);
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int pi = it * 8 + (pt >> 3);                 // (row, group) pair 0..63
+            const int r = pi & 15, grp = pi >> 4;
+            const int d0 = (grp >> 1) * 256 + static_cast<int>(rank) * 128 + (grp & 1) * 64;
+            // entry kk*16 + r of the block: register slot kk/2, lane (kk%2)*16 + r
+            const int v = __shfl_sync(0xffffffffu, cur[kk >> 1], (kk & 1) * 16 + r);
+            const uint16_t* src = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + d0 + c16 * 8;
+            cp_async16(dst0 + grp * 2048 + r * 128 + ((c16 ^ (r & 7)) << 4), src, v < 0 ? 0u : 16u);
+          }
+          cp_async_arrive_noinc(&S.v_loaded[st]);
+        }
       }
       cp_async_wait_all();
     } else if (warp == 9) {
       // ================================================================ relay
       // lane 0: S stages, lane 1: V stages.  Local completion -> the even CTA.
-      if (lane < 2) {
+      // lane 2: this CTA's 64 heads of Q (9 TMA boxes of 64 dims x 64 rows).
+      if (lane == 2) {
+        mbar_arrive_expect_tx(&S.q_full, kDChunks * kHalf * 128);
+        for (int dc = 0; dc < kDChunks; ++dc)
+          tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
+        if (mbar_wait(&S.q_full, 0, p.status, ab)) mbar_arrive_cluster(&S.q_ready, 0);
+      } else if (lane < 2) {
         const bool is_s = lane == 0;
         const int nchunks = is_s ? nblk * kDChunks : nblk * (kBlk / 16);
         const int stages = is_s ? kSStages : kVStages;
@@ -501,7 +534,9 @@ __global__ void __launch_bounds__(128) mla_combine_kernel(MlaParams p) {
 
 }  // namespace
 
-size_t mla_smem_bytes() { return sizeof(MlaSmem) + 1024; }
+static_assert(sizeof(MlaSmem) <= 232448, "sparse-MLA shared memory exceeds the 227 KB per-CTA limit");
+
+size_t mla_smem_bytes() { return sizeof(MlaSmem); }
 
 cudaError_t launch_sparse_mla(const MlaParams& p, const CUtensorMap& tm_q, cudaStream_t stream) {
   if (p.T == 0) return cudaSuccess;
