@@ -24,9 +24,12 @@
 // the rescale.  Rows are gathered by index with 16-byte cp.async (8 lanes per
 // 128-byte row segment: coalesced) into 128-byte-swizzled tiles.
 //
-// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-5 gather of the
-// S operand rows, 6-7 gather of the V operand rows, 8 TMEM owner and (in the
-// even CTA) MMA issuer, 9 relay.  Gather threads never wait for their own
+// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-7 gather of the
+// S operand rows, 8-11 gather of the V operand rows, 12 TMEM owner and (in
+// the even CTA) MMA issuer, 13-14 relays.  Signals from the odd CTA to the even
+// CTA's barriers are asynchronous 4-byte stores counted as transaction bytes
+// (a thread-level remote mbarrier arrive stalls its thread for a round trip,
+// which throttled the gathers to a fraction of the L2 bandwidth).  Gather threads never wait for their own
 // copies: each arrives on a local stage barrier through cp.async.mbarrier.arrive
 // (hardware-tracked completion), and a relay lane that has no copies in flight
 // forwards the completed stage to the even CTA's barrier, which the MMA issuer
@@ -40,7 +43,8 @@ namespace dsa {
 
 namespace {
 
-constexpr int kMlaThreads = 320;
+constexpr int kMlaThreads = 480;
+constexpr int kGatherWarps = 4;         // per operand ring; each warp loads whole chunks
 constexpr int kBlk = 128;             // selected rows per block (pair)
 constexpr int kHalf = 64;             // rows per CTA for the S operand; heads per CTA
 constexpr int kDChunks = DSA_D_QK / 64;   // 9 chunks of 64 dims
@@ -65,6 +69,8 @@ struct MlaSmem {
   uint64_t p_full, p_empty;
   uint64_t mx_bar[2], l_bar;
   uint64_t done;
+  // mailboxes of the peer CTA's asynchronous signals (contents unused)
+  uint32_t mbox_q, mbox_s[kSStages], mbox_v[kVStages], mbox_sfree[2][4], mbox_pfull[4];
   uint32_t tmem_base;
   int nblk, blk0;
   int abort_flag;
@@ -79,8 +85,11 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// No memory clobber: the copies are ordered against their consumers by mbarriers,
+// and leaving the compiler free to schedule address arithmetic keeps the gather
+// warps issuing back to back.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes));
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 // Arrive on `bar` once every cp.async issued so far by this thread has completed.
@@ -91,6 +100,19 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Cross-CTA signalling convention for barriers of the even CTA that wait on both
+// CTAs: the even CTA arrives locally (one arrival carrying expect_tx for the odd
+// CTA's bytes), the odd CTA sends 4-byte asynchronous stores (st_async_signal).
+__device__ __forceinline__ void pair_signal(uint32_t rank, uint64_t* bar, uint32_t* mbox, bool carries_tx,
+                                            uint32_t tx_bytes) {
+  if (rank == 0) {
+    if (carries_tx) mbar_arrive_expect_tx(bar, tx_bytes);
+    else mbar_arrive(bar);
+  } else {
+    st_async_signal(mbox, bar, 0, 1u);
+  }
 }
 
 // Lane-0 waits, the warp follows (warp-uniform result).
@@ -135,17 +157,17 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
 
   if (threadIdx.x == 0) {
     mbar_init(&S.q_full, 1);
-    mbar_init(&S.q_ready, 2);
+    mbar_init(&S.q_ready, 1);
     for (int i = 0; i < kSStages; ++i) {
-      mbar_init(&S.s_full[i], 2); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], 64);
+      mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], 32);
     }
     for (int i = 0; i < kVStages; ++i) {
-      mbar_init(&S.v_full[i], 2); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], 64);
+      mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], 32);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 8); mbar_init(&S.mx_bar[i], 128);
+      mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 4); mbar_init(&S.mx_bar[i], 128);
     }
-    mbar_init(&S.p_full, 8);
+    mbar_init(&S.p_full, 4);
     mbar_init(&S.p_empty, 1);
     mbar_init(&S.l_bar, 128);
     mbar_init(&S.done, 1);
@@ -181,7 +203,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       S.nblk = min(total, b0 + per) - b0;
     }
   }
-  if (warp == 8) tmem_alloc_pair(&S.tmem_base, 512);
+  if (warp == 12) tmem_alloc_pair(&S.tmem_base, 512);
   __syncwarp();
   tc_fence_before();
   cluster_sync_all();
@@ -220,7 +242,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(&S.s_free[sb], 0);
+        if (lane == 0) pair_signal(rank, &S.s_free[sb], &S.mbox_sfree[sb][warp], warp == 0, 16);
         float* x = reinterpret_cast<float*>(sr);             // logits in log2 units, in place
         float mloc = -INFINITY;
 #pragma unroll
@@ -279,7 +301,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(&S.p_full, 0);
+        if (lane == 0) pair_signal(rank, &S.p_full, &S.mbox_pfull[warp], warp == 0, 16);
       }
       // ---- epilogue: wait for the last PV, combine the two row halves, write out
       bool ok = !*ab;
@@ -335,134 +357,146 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
             p.part_lse[(static_cast<int64_t>(t) * p.splits + split) * H + h] = lse_v;
         }
       }
-    } else if (warp < 6) {
-      // ================================================================ S-operand gather
-      const int pt = threadIdx.x - 128;                      // 0..63
-      const int c16 = pt & 7;
-      // index entries of block j: lane holds entries 32*s + lane (s = 0..3), prefetched a block ahead
+    } else if (warp < 12) {
+      // ================================================================ gathers
+      // Warps 4-7 fill the S ring, warps 8-11 the V ring.  Chunk n of a ring is
+      // loaded entirely by warp n % 4 (16 copies of 16 B per lane, 8 lanes per
+      // 128-byte row segment) and signalled with one hardware-tracked arrive per
+      // lane.  Each warp keeps the local row indices of its current and next
+      // block in registers (lane l holds entries 32*s + l).
+      const bool is_s = warp < 8;
+      const int gw = (warp - 4) & 3;
+      const int per_blk = is_s ? kDChunks : kBlk / 16;
+      const int stages = is_s ? kSStages : kVStages;
+      const int n_total = nblk * per_blk;
+      uint64_t* empty = is_s ? S.s_empty : S.v_empty;
+      uint64_t* loaded = is_s ? S.s_loaded : S.v_loaded;
+      const int c16 = lane & 7;
       int cur[4], nxt[4];
+      int cur_blk = 0;
       block_rows(p, idx_row, blk0, len, lane, cur);
       if (nblk > 1) block_rows(p, idx_row, blk0 + 1, len, lane, nxt);
-      bool ok = true;
-      int n = 0;
-      for (int j = 0; j < nblk && ok; ++j) {
-        if (j > 0) {
+      for (int n = gw; n < n_total; n += kGatherWarps) {
+        const int j = n / per_blk, c = n % per_blk, st = n % stages;
+        while (cur_blk < j) {                                 // advance to block j (at most a few steps)
 #pragma unroll
           for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
-          if (j + 1 < nblk) block_rows(p, idx_row, blk0 + j + 1, len, lane, nxt);
+          ++cur_blk;
+          if (cur_blk + 1 < nblk) block_rows(p, idx_row, blk0 + cur_blk + 1, len, lane, nxt);
         }
-        for (int dc = 0; dc < kDChunks; ++dc, ++n) {
-          const int st = n % kSStages;
-          if (!warp_wait(&S.s_empty[st], ((n / kSStages) & 1) ^ 1, p.status, ab, false)) { ok = false; break; }
+        if (!warp_wait(&empty[st], ((n / stages) & 1) ^ 1, p.status, ab, false)) break;
+        const uint16_t* src[16];
+        uint32_t dst[16], nb[16];
+        if (is_s) {
           const uint32_t dst0 = smem_u32(S.s_ring[st]);
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int r = it * 8 + (pt >> 3);                  // row within this CTA's 64
-            // entry rank*64 + r of the block: register slot rank*2 + it/4, lane (it%4)*8 + pt/8
-            const int mine = rank ? cur[2 + (it >> 2)] : cur[it >> 2];
-            const int v = __shfl_sync(0xffffffffu, mine, (it & 3) * 8 + (pt >> 3));
-            const uint16_t* src = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + dc * 64 + c16 * 8;
-            cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4), src, v < 0 ? 0u : 16u);
+          for (int it = 0; it < 16; ++it) {
+            const int r = it * 4 + (lane >> 3);                // row within this CTA's 64
+            // entry rank*64 + r: register slot rank*2 + it/8, lane (it%8)*4 + lane/8
+            const int mine = rank ? cur[2 + (it >> 3)] : cur[it >> 3];
+            const int v = __shfl_sync(0xffffffffu, mine, (it & 7) * 4 + (lane >> 3));
+            src[it] = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + c * 64 + c16 * 8;
+            dst[it] = dst0 + r * 128 + ((c16 ^ (r & 7)) << 4);
+            nb[it] = v < 0 ? 0u : 16u;
           }
-          cp_async_arrive_noinc(&S.s_loaded[st]);
-        }
-      }
-      cp_async_wait_all();
-    } else if (warp < 8) {
-      // ================================================================ V-operand gather
-      const int pt = threadIdx.x - 192;                      // 0..63
-      const int c16 = pt & 7;
-      int cur[4], nxt[4];
-      block_rows(p, idx_row, blk0, len, lane, cur);
-      if (nblk > 1) block_rows(p, idx_row, blk0 + 1, len, lane, nxt);
-      bool ok = true;
-      int n = 0;
-      for (int j = 0; j < nblk && ok; ++j) {
-        if (j > 0) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
-          if (j + 1 < nblk) block_rows(p, idx_row, blk0 + j + 1, len, lane, nxt);
-        }
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk, ++n) {
-          const int st = n % kVStages;
-          if (!warp_wait(&S.v_empty[st], ((n / kVStages) & 1) ^ 1, p.status, ab, false)) { ok = false; break; }
+        } else {
           const uint32_t dst0 = smem_u32(S.v_ring[st]);
+          int mine = cur[0];
 #pragma unroll
-          for (int it = 0; it < 8; ++it) {
-            const int pi = it * 8 + (pt >> 3);                 // (row, group) pair 0..63
+          for (int u = 1; u < 4; ++u)
+            if ((c >> 1) == u) mine = cur[u];                  // register slot c/2 (warp-uniform)
+#pragma unroll
+          for (int it = 0; it < 16; ++it) {
+            const int pi = it * 4 + (lane >> 3);               // (row, group) pair 0..63
             const int r = pi & 15, grp = pi >> 4;
             const int d0 = (grp >> 1) * 256 + static_cast<int>(rank) * 128 + (grp & 1) * 64;
-            // entry kk*16 + r of the block: register slot kk/2, lane (kk%2)*16 + r
-            const int v = __shfl_sync(0xffffffffu, cur[kk >> 1], (kk & 1) * 16 + r);
-            const uint16_t* src = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + d0 + c16 * 8;
-            cp_async16(dst0 + grp * 2048 + r * 128 + ((c16 ^ (r & 7)) << 4), src, v < 0 ? 0u : 16u);
+            // entry c*16 + r of the block: register slot c/2, lane (c%2)*16 + r
+            const int v = __shfl_sync(0xffffffffu, mine, (c & 1) * 16 + r);
+            src[it] = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + d0 + c16 * 8;
+            dst[it] = dst0 + grp * 2048 + r * 128 + ((c16 ^ (r & 7)) << 4);
+            nb[it] = v < 0 ? 0u : 16u;
           }
-          cp_async_arrive_noinc(&S.v_loaded[st]);
         }
+#pragma unroll
+        for (int it = 0; it < 16; ++it) cp_async16(dst[it], src[it], nb[it]);
+        cp_async_arrive_noinc(&loaded[st]);
       }
       cp_async_wait_all();
-    } else if (warp == 9) {
-      // ================================================================ relay
-      // lane 0: S stages, lane 1: V stages.  Local completion -> the even CTA.
-      // lane 2: this CTA's 64 heads of Q (9 TMA boxes of 64 dims x 64 rows).
-      if (lane == 2) {
-        mbar_arrive_expect_tx(&S.q_full, kDChunks * kHalf * 128);
-        for (int dc = 0; dc < kDChunks; ++dc)
-          tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
-        if (mbar_wait(&S.q_full, 0, p.status, ab)) mbar_arrive_cluster(&S.q_ready, 0);
-      } else if (lane < 2) {
-        const bool is_s = lane == 0;
-        const int nchunks = is_s ? nblk * kDChunks : nblk * (kBlk / 16);
+    } else if (warp >= 13) {
+      // ================================================================ relays
+      // Warp 13 lane 0: this CTA's Q load (9 TMA boxes of 64 dims x 64 heads) and
+      // the S ring; warp 14 lane 0: the V ring.  Each forwards completed stages,
+      // in order, to the even CTA's barriers.  They wait with the suspending
+      // try_wait: a spinning test_wait poller competes with the gathers for the
+      // shared-memory pipe.  As in cp.async-fed tensor-core pipelines, the stage
+      // barrier (completed by the copies themselves) orders the data before the
+      // MMA that reads it, so no proxy fence is issued here.
+      if (lane == 0) {
+        const bool is_s = warp == 13;
+        if (is_s) {
+          mbar_arrive_expect_tx(&S.q_full, kDChunks * kHalf * 128);
+          for (int dc = 0; dc < kDChunks; ++dc)
+            tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
+          if (mbar_wait(&S.q_full, 0, p.status, ab)) pair_signal(rank, &S.q_ready, &S.mbox_q, true, 4);
+        }
+        const int n = nblk * (is_s ? kDChunks : kBlk / 16);
         const int stages = is_s ? kSStages : kVStages;
         uint64_t* loaded = is_s ? S.s_loaded : S.v_loaded;
         uint64_t* full = is_s ? S.s_full : S.v_full;
-        for (int n = 0; n < nchunks; ++n) {
-          const int st = n % stages;
-          if (!mbar_wait(&loaded[st], (n / stages) & 1, p.status, ab)) break;
-          fence_proxy_async_smem();
-          mbar_arrive_cluster(&full[st], 0);
+        uint32_t* mbox = is_s ? S.mbox_s : S.mbox_v;
+        for (int i = 0; i < n; ++i) {
+          const int st = i % stages;
+          if (!mbar_wait(&loaded[st], (i / stages) & 1, p.status, ab)) break;
+          pair_signal(rank, &full[st], &mbox[st], true, 4);
         }
       }
     } else if (rank == 0 && lane == 0) {
       // ================================================================ MMA issuer (even CTA)
+      // Waits use the CTA-scope try_wait, as 2-SM tensor-core pipelines do for the
+      // leader's stage barriers: a cluster-scope acquire on every stage cost about
+      // 0.35 us each and throttled MMA issue.
       const uint32_t id_s = instr_desc(1, 1, false, false, 128, kBlk);   // bf16 x bf16, M=128 pair, N=128
       const uint32_t id_pv = instr_desc(1, 1, false, true, 128, 256);    // B (V) MN-major, N=256
-      bool ok = mbar_wait_cluster(&S.q_ready, 0, p.status, ab);
-      int sc = 0, vc = 0;
+      bool ok = mbar_wait(&S.q_ready, 0, p.status, ab);
+      // Descriptors are built once; a step inside a tile adds to the 14-bit
+      // start-address field (16-byte units).  Each ring holds exactly one block,
+      // so chunk c of every block sits in slot c and is in its (block)-th phase.
+      static_assert(kSStages == kDChunks && kVStages == kBlk / 16, "one block per ring");
+      const uint64_t qd0 = smem_desc_sw128(smem_u32(S.q[0]), 16, 1024);
+      const uint64_t sd0 = smem_desc_sw128(smem_u32(S.s_ring[0]), 16, 1024);
+      const uint64_t pd0 = smem_desc_sw128(smem_u32(S.p[0]), 16, 1024);
+      const uint64_t vd0 = smem_desc_sw128(smem_u32(S.v_ring[0]), 2048, 1024);
       auto issue_s = [&](int j) -> bool {
         const int sb = j & 1;
-        if (!mbar_wait_cluster(&S.s_free[sb], ((j >> 1) & 1) ^ 1, p.status, ab)) return false;
+        if (!mbar_wait(&S.s_free[sb], ((j >> 1) & 1) ^ 1, p.status, ab)) return false;
         tc_fence_after();
-        for (int dc = 0; dc < kDChunks; ++dc, ++sc) {
-          const int st = sc % kSStages;
-          if (!mbar_wait_cluster(&S.s_full[st], (sc / kSStages) & 1, p.status, ab)) return false;
+        const uint32_t d = tmem + kSCol + sb * 64;
+#pragma unroll
+        for (int dc = 0; dc < kDChunks; ++dc) {
+          if (!mbar_wait(&S.s_full[dc], j & 1, p.status, ab)) return false;
           tc_fence_after();
-          const uint32_t qa = smem_u32(S.q[dc]);
-          const uint32_t sa = smem_u32(S.s_ring[st]);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_pair(tmem + kSCol + sb * 64, smem_desc_sw128(qa + kk * 32, 16, 1024),
-                           smem_desc_sw128(sa + kk * 32, 16, 1024), id_s, (dc | kk) != 0 ? 1u : 0u);
-          umma_commit_pair(&S.s_empty[st], 0x3);
+            umma_bf16_pair(d, qd0 + static_cast<uint64_t>(dc * (kHalf * 128 / 16) + kk * 2),
+                           sd0 + static_cast<uint64_t>(dc * (kHalf * 128 / 16) + kk * 2), id_s, (dc | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(&S.s_empty[dc], 0x3);
         }
         umma_commit_pair(&S.s_ready[sb], 0x3);
         return true;
       };
       auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait_cluster(&S.p_full, j & 1, p.status, ab)) return false;
+        if (!mbar_wait(&S.p_full, j & 1, p.status, ab)) return false;
         tc_fence_after();
-        for (int kk = 0; kk < kBlk / 16; ++kk, ++vc) {
-          const int st = vc % kVStages;
-          if (!mbar_wait_cluster(&S.v_full[st], (vc / kVStages) & 1, p.status, ab)) return false;
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          if (!mbar_wait(&S.v_full[kk], j & 1, p.status, ab)) return false;
           tc_fence_after();
-          const uint32_t pa = smem_u32(S.p[kk >> 2]) + (kk & 3) * 32;
-          const uint32_t va = smem_u32(S.v_ring[st]);
+          const uint64_t pa = pd0 + static_cast<uint64_t>((kk >> 2) * (kHalf * 128 / 16) + (kk & 3) * 2);
 #pragma unroll
           for (int c = 0; c < 2; ++c)
-            umma_bf16_pair(tmem + kOCol + c * 128, smem_desc_sw128(pa, 16, 1024),
-                           smem_desc_sw128(va + c * 4096, 2048, 1024), id_pv, (j | kk) != 0 ? 1u : 0u);
-          umma_commit_pair(&S.v_empty[st], 0x3);
+            umma_bf16_pair(tmem + kOCol + c * 128, pa, vd0 + static_cast<uint64_t>(kk * (4 * 16 * 128 / 16) + c * 256),
+                           id_pv, (j | kk) != 0 ? 1u : 0u);
+          umma_commit_pair(&S.v_empty[kk], 0x3);
         }
         umma_commit_pair(&S.p_empty, 0x3);
         return true;
@@ -500,7 +534,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
   __syncwarp();
   tc_fence_before();
   cluster_sync_all();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, 512);
   }
