@@ -147,6 +147,34 @@ dsa_status dsa_forward(const dsa_batch *batch, const uint8_t *q_idx, const uint8
                        float sm_scale, uint16_t *out, float *lse, void *ws, size_t ws_bytes,
                        void *stream);
 
+/*
+ * Lightning indexer scores for callers that cannot allocate device memory.
+ * The method has no counterpart for this entry point; it exists for
+ * integration: some callers cannot call cudaMalloc (a host framework that
+ * only hands out the tensors of the operation, a plug-in running inside
+ * someone else's memory pool, code between steps that must not grow the
+ * footprint), so they cannot provide the workspace `ws` that
+ * dsa_indexer_scores needs for its per-call plan and status word.
+ * This variant computes exactly what dsa_indexer_scores computes (same
+ * arguments and results, no ws) and keeps that scratch in a fixed device array
+ * inside the library instead:
+ *   - Limit: num_q <= DSA_NOALLOC_MAX_Q; larger batches return
+ *     DSA_ERR_UNSUPPORTED before anything is launched.  The array is about
+ *     400 KB and every GPU that loads the library holds it until the process
+ *     exits.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the array and leaves its contents behind;
+ *     calls whose kernels overlap on the GPU (e.g. on two streams) race on it,
+ *     so serialise them.
+ *   - Device-side flags (see DSA_DEV_*) land in the shared array and are not
+ *     reported; host-side argument errors are.
+ * Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define DSA_NOALLOC_MAX_Q 16384
+dsa_status dsa_indexer_scores_noalloc(const dsa_batch *batch, const uint8_t *q_idx, const uint8_t *k_idx,
+                                      const float *w, int H_I, float *scores, int64_t ld, void *stream);
+
 /* Pointers into a forward workspace (for inspection by tests): scores [T, ld]
  * fp32 and idx [T, k] int32.  Returns DSA_ERR_INVALID_ARGUMENT on bad input. */
 dsa_status dsa_forward_ws_views(const dsa_batch *batch, int H_I, int H, int k, void *ws,

@@ -24,7 +24,9 @@ DEV_BAD_QUERY, DEV_BAD_INDEX, DEV_TIMEOUT = 1, 2, 4
 OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD = 0, 1, 2, 3
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward",
-           "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version")
+           "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
+           "dsa_indexer_scores_noalloc")
+NOALLOC_MAX_Q = 16384
 
 
 class DsaError(RuntimeError):
@@ -62,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_topk.argtypes = [bp, vp, i64, i32, vp, vp, sz, vp]
         L.dsa_sparse_mla.argtypes = [bp, vp, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
         L.dsa_forward.argtypes = [bp, vp, vp, vp, i32, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
+        L.dsa_indexer_scores_noalloc.argtypes = [bp, vp, vp, vp, i32, vp, i64, vp]
         L.dsa_forward_ws_views.argtypes = [bp, i32, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(i64),
                                            ctypes.POINTER(vp)]
         L.dsa_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
@@ -69,7 +72,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = i32
         for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward", "dsa_forward_ws_views",
-                   "dsa_read_device_status"):
+                   "dsa_read_device_status", "dsa_indexer_scores_noalloc"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -140,6 +143,12 @@ def dsa_indexer_scores(batch: DeviceBatch, q_idx, k_idx, w, H_I: int, scores, ld
     _check("dsa_indexer_scores", lib().dsa_indexer_scores(
         ctypes.byref(batch.struct), _ptr(q_idx), _ptr(k_idx), _ptr(w), H_I, _ptr(scores), ld, _ptr(ws),
         ws.numel(), _stream(stream)))
+
+
+def dsa_indexer_scores_noalloc(batch: DeviceBatch, q_idx, k_idx, w, H_I: int, scores, ld: int, stream=None):
+    """dsa_indexer_scores without a workspace (scratch in a fixed device array of the library)."""
+    _check("dsa_indexer_scores_noalloc", lib().dsa_indexer_scores_noalloc(
+        ctypes.byref(batch.struct), _ptr(q_idx), _ptr(k_idx), _ptr(w), H_I, _ptr(scores), ld, _stream(stream)))
 
 
 def dsa_topk(batch: DeviceBatch, scores, ld: int, k: int, idx, ws, stream=None):

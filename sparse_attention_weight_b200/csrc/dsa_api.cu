@@ -331,3 +331,48 @@ const char* dsa_status_string(dsa_status s) {
 int dsa_abi_version(void) { return DSA_ABI_VERSION; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Indexer without a caller workspace: the plan and status word live in a
+// fixed device array of this file (sized for DSA_NOALLOC_MAX_Q queries).
+namespace {
+constexpr size_t kNoAllocBytes = kWsHeader + (6 * static_cast<size_t>(DSA_NOALLOC_MAX_Q) + 2) * sizeof(int32_t);
+}  // namespace
+
+// In host code this name stands for the array, not for a device address; the
+// kernels get the address that cudaGetSymbolAddress returns on each device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
+
+namespace {
+void* noalloc_scratch_on_current_device() {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    addr[dev] = p;
+  }
+  return addr[dev];
+}
+}  // namespace
+
+extern "C" dsa_status dsa_indexer_scores_noalloc(const dsa_batch* batch, const uint8_t* q_idx,
+                                                 const uint8_t* k_idx, const float* w, int H_I, float* scores,
+                                                 int64_t ld, void* stream) {
+  if (!batch_ok(batch)) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!q_idx || !k_idx || !w || !scores)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!hi_ok(H_I)) return DSA_ERR_UNSUPPORTED;
+  if (batch->num_q > DSA_NOALLOC_MAX_Q) return DSA_ERR_UNSUPPORTED;
+  if (ld < batch->max_kv_len || ld % 4 != 0) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(scores)) return DSA_ERR_UNSUPPORTED;
+  void* ws = noalloc_scratch_on_current_device();
+  if (!ws) return DSA_ERR_CUDA;
+  const WsLayout L = layout(ws, DSA_OP_INDEXER, batch, 8, 1, ld);
+  if (L.bytes > kNoAllocBytes) return DSA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;   // starts at zero
+  return run_indexer(batch, q_idx, k_idx, w, H_I, scores, ld, L, st);
+}
