@@ -39,6 +39,11 @@ from sparse_attention_weight_b200.configs import WORKLOADS  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20
 MLA_FLOP_PER_PAIR = 128 * (576 + 512) * 2       # per (query, selected row) at H = 128
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
+# (profiles/sparse_mla_prefill_L2304.md: 624.0 MB at 2304 queries), scaled by the
+# number of queries (the traffic is the queries in and the outputs out; the cache
+# gathers hit L2).  None where no capture stands for the current kernel.
+MLA_TRAFFIC_BYTES_PER_QUERY = 624.0e6 / 2304
 IDX_FLOP_PER_PAIR = 64 * 128 * 2                # per (query, visible key) at H_I = 64
 
 
@@ -342,7 +347,7 @@ def main():
                 "unit": "TFLOP/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["peak_source"] = peaks["src"] + (" (burst)" if roof["unit"] == "TFLOP/s" else "")
-    roof["traffic"] = None
+    roof["traffic"] = (MLA_TRAFFIC_BYTES_PER_QUERY * T) if wl.kind == "prefill" else None
     idx_tflops = res["idx_pairs"] * IDX_FLOP_PER_PAIR * wl.h_index / 64 / (idx_ms / 1e3) / 1e12
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,

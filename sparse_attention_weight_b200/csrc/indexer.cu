@@ -97,11 +97,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         int g = find_group(p.item_off, ngroups, i0);
         int g_lo = p.item_off[g], g_hi = p.item_off[g + 1];
         int prev_g = -1, issued = 0, q_loads = 0;
+        int64_t row_base = 0;                   // first cache row of the group's sequence
         uint32_t qe_par = 0;
         for (int i = i0; i < i1; ++i) {
           while (g_hi <= i) { ++g; g_lo = g_hi; g_hi = p.item_off[g + 1]; }
           const int kt = i - g_lo;
           if (g != prev_g) {
+            row_base = p.kv_offset[p.group_seq[g]];
             if (prev_g >= 0) {
               if (!mbar_wait(&S.q_empty, qe_par, p.status, abort_flag)) break;
               qe_par ^= 1;
@@ -115,7 +117,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint32_t ph = (n / kStages) & 1;
           if (!mbar_wait(&S.k_empty[st], ph ^ 1, p.status, abort_flag)) break;
           mbar_arrive_expect_tx(&S.k_full[st], kTileBytes);
-          const int64_t row = p.kv_offset[p.group_seq[g]] + static_cast<int64_t>(kt) * kKeyTile;
+          const int64_t row = row_base + static_cast<int64_t>(kt) * kKeyTile;
           tma_load_2d(S.k[st], &tm_k, &S.k_full[st], 0, static_cast<int>(row));
           ++issued;
         }
