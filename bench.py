@@ -119,6 +119,29 @@ def _smi_index(local: int) -> int:
     return local
 
 
+def reduce_max(value: float, device=None) -> float:
+    """Max of `value` over the ranks of the default process group (identity when
+    there is none); used for the timed region, which is reported as the max over
+    ranks."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return units_per_rank * world / (ms / 1e3)
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own shard: the same workload drawn from its own seed."""
+    return rank
+
+
 def _algorithmic(wl, batch, idx_host=None):
     """Algorithmic work of one step: indexer (query, visible key) pairs and
     sparse-MLA (query, selected row) pairs; selected rows = min(n_t, k)."""
@@ -135,7 +158,7 @@ def run_ours(args, wl, rank, world, device):
     from sparse_attention_weight_b200 import inputs
 
     chunk = (wl.seq_len // wl.chunk - 1) if wl.kind == "chunked_prefill" else None
-    ins = inputs.make_inputs(wl, seed=rank, chunk_index=chunk)
+    ins = inputs.make_inputs(wl, seed=rank_seed(rank), chunk_index=chunk)
     bh = ins["batch"]
     T = bh.num_q
     B.lib()
@@ -187,11 +210,7 @@ def run_ours(args, wl, rank, world, device):
     if world > 1:
         torch.distributed.barrier()
     stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in events])   # ms
-    total_ms = float(stage.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(float(stage.sum()), device)
     ms_per_step = total_ms / args.steps
     idx_pairs, sel_pairs = _algorithmic(wl, bh)
 
@@ -223,12 +242,8 @@ def run_ours(args, wl, rank, world, device):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": T * world / (e2e_ms / 1e3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+        e2e_ms = reduce_max(e0.elapsed_time(e1) / n_e2e, device)
+        e2e = {"value": whole_job_rate(T, world, e2e_ms), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms}
     splits = 1
     try:
@@ -333,7 +348,7 @@ def main():
     res = run_ours(args, wl, rank, world, device)
     peaks = _peaks()
     T = res["T"]
-    value = T * world / (res["ms_per_step"] / 1e3)
+    value = whole_job_rate(T, world, res["ms_per_step"])
     st = res["stage_ms"]
     mla_ms, idx_ms, topk_ms = st[2], st[0], st[1]
     mla_tflops = res["sel_pairs"] * MLA_FLOP_PER_PAIR * wl.heads / 128 / (mla_ms / 1e3) / 1e12

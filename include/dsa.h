@@ -186,6 +186,15 @@ dsa_status dsa_forward_ws_views(const dsa_batch *batch, int H_I, int H, int k, v
  */
 dsa_status dsa_read_device_status(const void *ws, uint32_t *flags, void *stream);
 
+/*
+ * Self-test of the bounded waits that guard every in-kernel spin wait, i.e. of
+ * failure detection without faulting a GPU: one thread waits on a barrier that
+ * nothing completes, gives up after `limit_us` microseconds (1 .. 2,000,000),
+ * records DSA_DEV_TIMEOUT in the status word of `ws` (>= 256 bytes) and returns;
+ * the context stays usable.  Read the flag with dsa_read_device_status.
+ */
+dsa_status dsa_selftest_wait_timeout(void *ws, size_t ws_bytes, uint32_t limit_us, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *dsa_status_string(dsa_status status);
 

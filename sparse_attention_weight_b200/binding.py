@@ -25,7 +25,7 @@ OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD = 0, 1, 2, 3
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward",
            "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
-           "dsa_indexer_scores_noalloc")
+           "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout")
 NOALLOC_MAX_Q = 16384
 
 
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_mla.argtypes = [bp, vp, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
         L.dsa_forward.argtypes = [bp, vp, vp, vp, i32, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
         L.dsa_indexer_scores_noalloc.argtypes = [bp, vp, vp, vp, i32, vp, i64, vp]
+        L.dsa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
         L.dsa_forward_ws_views.argtypes = [bp, i32, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(i64),
                                            ctypes.POINTER(vp)]
         L.dsa_read_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
@@ -72,7 +73,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = i32
         for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward", "dsa_forward_ws_views",
-                   "dsa_read_device_status", "dsa_indexer_scores_noalloc"):
+                   "dsa_read_device_status", "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -176,6 +177,11 @@ def forward_ws_views(batch: DeviceBatch, H_I: int, H: int, k: int, ws) -> tuple[
     _check("dsa_forward_ws_views", lib().dsa_forward_ws_views(ctypes.byref(batch.struct), H_I, H, k, _ptr(ws),
                                                               ctypes.byref(s), ctypes.byref(ld), ctypes.byref(i)))
     return s.value, ld.value, i.value
+
+
+def dsa_selftest_wait_timeout(ws, limit_us: int, stream=None):
+    _check("dsa_selftest_wait_timeout", lib().dsa_selftest_wait_timeout(_ptr(ws), ws.numel(), limit_us,
+                                                                        _stream(stream)))
 
 
 def read_device_status(ws, stream=None) -> int:

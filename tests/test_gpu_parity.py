@@ -309,3 +309,23 @@ def test_device_status_flags_bad_queries_and_indices(cuda_device):
     ws3 = B.workspace(B.OP_SPARSE_MLA, good["batch"], H=128, k=wl.k, device=cuda_device)
     B.dsa_sparse_mla(good["batch"], good["q"], good["kv"], i_dev, wl.k, 128, wl.sm_scale, out, None, ws3)
     assert B.read_device_status(ws3) & B.DEV_BAD_INDEX
+
+
+# ----------------------------------------------------------------------------- failure detection
+
+
+def test_bounded_wait_times_out_and_leaves_the_context_usable(cuda_device):
+    """A barrier that nothing completes: the waiting kernel gives up after the
+    limit, flags DSA_DEV_TIMEOUT, and later work on the same context runs."""
+    import time
+    ws = torch.zeros(256, dtype=torch.uint8, device=cuda_device)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    B.dsa_selftest_wait_timeout(ws, 20000)          # 20 ms
+    flags = B.read_device_status(ws)
+    dt = time.perf_counter() - t0
+    assert flags & B.DEV_TIMEOUT
+    assert 0.015 < dt < 5.0
+    x = torch.arange(10, device=cuda_device).sum().item()
+    assert x == 45
+    _topk_case(cuda_device, [np.arange(300, dtype=np.float32)], 64)
