@@ -119,16 +119,21 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // Wait for phase `parity` of `bar` to complete.  Returns false (and records
 // DSA_DEV_TIMEOUT, and sets *abort) if it did not complete within `limit_ns`
 // or if another thread of the CTA already aborted.
+// Reading %globaltimer costs a few hundred nanoseconds, so the clock is started
+// only after 1024 unsuccessful polls and read once per 1024 polls after that: a
+// wait that completes soon never touches it.
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, uint32_t* status,
                                                 volatile int* abort_flag, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((it & 63u) == 0) {
+    if ((it & 1023u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
         set_status(status, DSA_DEV_TIMEOUT);
         if (abort_flag) *abort_flag = 1;
         return false;
@@ -145,13 +150,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t* status,
                                                   volatile int* abort_flag) {
   const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait_cluster(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_cluster(a, parity)) return true;
-    if ((it & 63u) == 0) {
+    if ((it & 1023u) == 0) {
       if (abort_flag && *abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
         set_status(status, DSA_DEV_TIMEOUT);
         if (abort_flag) *abort_flag = 1;
         return false;
