@@ -181,6 +181,15 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// 2^x on the special-function unit (PTX ex2.approx.ftz: relative error about
+// 2^-22, subnormal results flushed to zero, 2^-inf = 0).  The softmax feeds its
+// results to bf16, so the approximation is far below the rounding it gets.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---------------------------------------------------------------- TMA
 // 2-D tiled load: coordinates (x = innermost, in elements; y = row).
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,

@@ -72,7 +72,7 @@ struct MlaSmem {
   // mailboxes of the peer CTA's asynchronous signals (contents unused)
   uint32_t mbox_q, mbox_s[kSStages], mbox_v[kVStages], mbox_sfree[2][4], mbox_pfull[4];
   uint32_t tmem_base;
-  int nblk, blk0;
+  int last_used[8];                          // per prologue warp: last usable entry, -1 if none
   int abort_flag;
 };
 
@@ -179,29 +179,28 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
     fence_mbar_init();
     if (!rows_ok) set_status(p.status, DSA_DEV_BAD_QUERY);
   }
-  // blocks of 128 entries covering the used part of the index row, split evenly
-  if (warp == 4) {
+  // Validity bitmask of the index row: warps 4-11 take 8 words (256 entries)
+  // each, all loads in flight at once; each records its last usable entry.
+  if (warp >= 4 && warp < 12) {
+    const int w8 = warp - 4;
+    int v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = (w8 * 8 + u) * 32 + lane;
+      v[u] = (rows_ok && i < p.k) ? __ldg(idx_row + i) : -1;
+    }
     int last = -1;
-    for (int b = 0; b < 2048 / 32; ++b) {
-      const int i = b * 32 + lane;
-      int v = -1;
-      if (rows_ok && i < p.k) {
-        v = __ldg(idx_row + i);
-        if (v >= len) { set_status(p.status, DSA_DEV_BAD_INDEX); v = -1; }
-      }
-      if (v >= 0) last = i;
-      const uint32_t m = __ballot_sync(0xffffffffu, v >= 0);
-      if (lane == 0) S.valid[b] = m;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = (w8 * 8 + u) * 32 + lane;
+      if (v[u] >= len) { set_status(p.status, DSA_DEV_BAD_INDEX); v[u] = -1; }
+      if (v[u] >= 0) last = i;
+      const uint32_t m = __ballot_sync(0xffffffffu, v[u] >= 0);
+      if (lane == 0) S.valid[w8 * 8 + u] = m;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-    if (lane == 0) {
-      const int total = (last + kBlk) / kBlk;
-      const int per = (total + p.splits - 1) / p.splits;
-      const int b0 = min(total, split * per);
-      S.blk0 = b0;
-      S.nblk = min(total, b0 + per) - b0;
-    }
+    if (lane == 0) S.last_used[w8] = last;
   }
   if (warp == 12) tmem_alloc_pair(&S.tmem_base, 512);
   __syncwarp();
@@ -209,8 +208,17 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
-  const int nblk = S.abort_flag ? 0 : S.nblk;
-  const int blk0 = S.blk0;
+  // blocks of 128 entries covering the used part of the index row, split evenly
+  int nblk = 0, blk0 = 0;
+  {
+    int last = -1;
+#pragma unroll
+    for (int w8 = 0; w8 < 8; ++w8) last = max(last, S.last_used[w8]);
+    const int total = (last + kBlk) / kBlk;
+    const int per = (total + p.splits - 1) / p.splits;
+    blk0 = min(total, split * per);
+    nblk = S.abort_flag ? 0 : min(total, blk0 + per) - blk0;
+  }
 
   const int H = p.H;
   const int head0 = static_cast<int>(rank) * kHalf;        // first head of this CTA
@@ -258,16 +266,19 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         const float mblk = fmaxf(mloc, S.xmax[sb][tid ^ 64]);
         const bool rescale = mblk > m_ref + kRescaleThreshold;
         const float m_new = rescale ? mblk : m_ref;
+        // a head with no usable entry so far has m_new = -inf and every x = -inf:
+        // subtract 0 instead, so that each p is 2^-inf = 0 (never -inf - -inf)
+        const float msub = m_new == -INFINITY ? 0.f : m_new;
         float psum = 0.f;
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          const float p0 = x[c] == -INFINITY ? 0.f : exp2f(x[c] - m_new);
-          const float p1 = x[c + 1] == -INFINITY ? 0.f : exp2f(x[c + 1] - m_new);
+          const float p0 = ex2_approx(x[c] - msub);
+          const float p1 = ex2_approx(x[c + 1] - msub);
           psum += p0 + p1;
           pk[c >> 1] = pack_bf16(p0, p1);
         }
-        const float alpha = rescale ? exp2f(m_ref - m_new) : 1.f;   // m_ref = -inf -> 0
+        const float alpha = rescale ? ex2_approx(m_ref - m_new) : 1.f;   // m_ref = -inf -> 0
         l = l * alpha + psum;
         // P buffer and O are free once PV of the previous block completed
         if (j > 0) {
