@@ -21,19 +21,25 @@
 // while the softmax warps turn S of block j into P.  The softmax keeps a
 // reference maximum per head and rescales O (in TMEM) only when a block's
 // maximum exceeds it by more than 2^8, so P stays <= 256 and most blocks skip
-// the rescale.  Rows are gathered by index with 16-byte cp.async (8 lanes per
-// 128-byte row segment: coalesced) into 128-byte-swizzled tiles.
+// the rescale.  Rows are gathered from L2 by index with 16-byte cp.async (8
+// lanes per 128-byte row segment: coalesced) into 128-byte-swizzled tiles, once:
+// each CTA gathers its 64 rows x 576 dims for S, and the V operand (the first
+// 512 of those dims, needed by both CTAs, each for its value dims) is copied
+// out of the S rings by bulk shared-memory copies across the pair.  Gathering
+// V from L2 a second time nearly doubled the gather traffic, and the gathers'
+// latency, not the tensor core, set the pace.
 //
-// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-7 gather of the
-// S operand rows, 8-11 gather of the V operand rows, 12 TMEM owner and (in
-// the even CTA) MMA issuer, 13-14 relays.  Signals from the odd CTA to the even
-// CTA's barriers are asynchronous 4-byte stores counted as transaction bytes
-// (a thread-level remote mbarrier arrive stalls its thread for a round trip,
-// which throttled the gathers to a fraction of the L2 bandwidth).  Gather threads never wait for their own
-// copies: each arrives on a local stage barrier through cp.async.mbarrier.arrive
-// (hardware-tracked completion), and a relay lane that has no copies in flight
-// forwards the completed stage to the even CTA's barrier, which the MMA issuer
-// waits on.
+// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-11 gather of the
+// S operand rows, 12 TMEM owner and (in the even CTA) issuer of the S MMAs,
+// 13 Q load and S relay, 14 V copier and relay, 15 (even CTA) issuer of the
+// PV MMAs.  Signals from the odd CTA to the even CTA's barriers are
+// asynchronous 4-byte stores counted as transaction bytes (a thread-level
+// remote mbarrier arrive stalls its thread for a round trip, which throttled
+// the gathers when every stage used one).  Gather threads never wait for their
+// own copies: each arrives on a local stage barrier through
+// cp.async.mbarrier.arrive (hardware-tracked completion), and a relay lane
+// that has no copies in flight forwards the completed stage to the even CTA's
+// barrier, which the MMA issuer waits on.
 #include <cuda_bf16.h>
 
 #include "dsa_common.cuh"
@@ -43,13 +49,13 @@ namespace dsa {
 
 namespace {
 
-constexpr int kMlaThreads = 480;
-constexpr int kGatherWarps = 4;         // per operand ring; each warp loads whole chunks
+constexpr int kMlaThreads = 512;
+constexpr int kGatherWarps = 8;         // S-ring gather warps; each warp loads whole chunks
 constexpr int kBlk = 128;             // selected rows per block (pair)
 constexpr int kHalf = 64;             // rows per CTA for the S operand; heads per CTA
 constexpr int kDChunks = DSA_D_QK / 64;   // 9 chunks of 64 dims
 constexpr int kSStages = 9;           // S-operand ring (8 KB slots): one full block
-constexpr int kVStages = 8;           // V-operand ring (8 KB slots): one full block
+constexpr int kVChunks = 8;           // value dims 0..511 = S-ring chunks 0..7
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr uint32_t kSCol = 0;         // TMEM columns [0,128): two S buffers of 64
 constexpr uint32_t kOCol = 128;       // TMEM columns [128,384): O (2 x 128)
@@ -57,20 +63,21 @@ constexpr uint32_t kOCol = 128;       // TMEM columns [128,384): O (2 x 128)
 struct MlaSmem {
   uint8_t q[kDChunks][kHalf * 128];          // 72 KB  Q of this CTA's heads (K-major SW128)
   uint8_t s_ring[kSStages][kHalf * 128];     // 64 KB  S operand chunks: 64 rows x 64 dims
-  uint8_t v_ring[kVStages][4][16 * 128];     // 48 KB  V operand chunks: 16 rows x 4 dim groups
+  uint8_t vbuf[4][kBlk * 128];               // 64 KB  V operand: 4 dim groups x 128 rows (MN-major SW128)
   uint8_t p[2][kHalf * 128];                 // 16 KB  P: 64 heads x 128 rows (two K chunks)
   float xmax[2][128];
   float lsum[128];
   uint32_t valid[2048 / 32];                 // bit e: entry e of the index row is a usable row
   uint64_t q_full, q_ready;
   uint64_t s_full[kSStages], s_empty[kSStages], s_loaded[kSStages];
-  uint64_t v_full[kVStages], v_empty[kVStages], v_loaded[kVStages];
+  uint64_t v_full[2], v_empty[2], v_loaded[2];   // per half of the block's rows (= per CTA's rows)
+  uint64_t xfer;                             // this CTA's copies of a block into both V buffers landed
   uint64_t s_ready[2], s_free[2];
   uint64_t p_full, p_empty;
   uint64_t mx_bar[2], l_bar;
   uint64_t done;
   // mailboxes of the peer CTA's asynchronous signals (contents unused)
-  uint32_t mbox_q, mbox_s[kSStages], mbox_v[kVStages], mbox_sfree[2][4], mbox_pfull[4];
+  uint32_t mbox_q, mbox_s[kSStages], mbox_v[2], mbox_sfree[2][4], mbox_pfull[4];
   uint32_t tmem_base;
   int last_used[8];                          // per prologue warp: last usable entry, -1 if none
   int abort_flag;
@@ -95,6 +102,22 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // Arrive on `bar` once every cp.async issued so far by this thread has completed.
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Address of the same shared-memory object in CTA `cta` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(cta));
+  return r;
+}
+
+// Bulk copy of `bytes` from this CTA's shared memory to `dst`, a shared::cluster
+// address in this CTA or its peer; the bytes are counted on `bar`, a barrier in
+// the destination CTA.
+__device__ __forceinline__ void bulk_copy_s2c(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -161,16 +184,17 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
     for (int i = 0; i < kSStages; ++i) {
       mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], 32);
     }
-    for (int i = 0; i < kVStages; ++i) {
-      mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], 1);
     }
+    mbar_init(&S.xfer, 2);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 4); mbar_init(&S.mx_bar[i], 128);
     }
     mbar_init(&S.p_full, 4);
     mbar_init(&S.p_empty, 1);
     mbar_init(&S.l_bar, 128);
-    mbar_init(&S.done, 1);
+    mbar_init(&S.done, 2);                      // one drain commit per MMA issuer
     S.abort_flag = 0;
     if (smem_u32(smem_raw) & 1023u) {           // the swizzled tiles need 1024-byte alignment
       set_status(p.status, DSA_DEV_INTERNAL);
@@ -370,113 +394,126 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       }
     } else if (warp < 12) {
       // ================================================================ gathers
-      // Warps 4-7 fill the S ring, warps 8-11 the V ring.  Chunk n of a ring is
-      // loaded entirely by warp n % 4 (16 copies of 16 B per lane, 8 lanes per
-      // 128-byte row segment) and signalled with one hardware-tracked arrive per
-      // lane.  Each warp keeps the local row indices of its current and next
-      // block in registers (lane l holds entries 32*s + l).
-      const bool is_s = warp < 8;
-      const int gw = (warp - 4) & 3;
-      const int per_blk = is_s ? kDChunks : kBlk / 16;
-      const int stages = is_s ? kSStages : kVStages;
-      const int n_total = nblk * per_blk;
-      uint64_t* empty = is_s ? S.s_empty : S.v_empty;
-      uint64_t* loaded = is_s ? S.s_loaded : S.v_loaded;
+      // Warps 4-11 fill the S ring: chunk n (dims 64c..64c+63 of this CTA's 64
+      // rows of block n / 9) is loaded entirely by warp n % 8 (16 copies of 16 B
+      // per lane, 8 lanes per 128-byte row segment) and signalled with one
+      // hardware-tracked arrive per lane.  A slot is refilled once the S MMA read
+      // it and, for value chunks, once its copies into the V buffers landed.
+      // Each warp keeps the local row indices of its current and next block in
+      // registers (lane l holds entries 32*s + l).
+      const int gw = warp - 4;
+      const int n_total = nblk * kDChunks;
       const int c16 = lane & 7;
       int cur[4], nxt[4];
       int cur_blk = 0;
       block_rows(p, idx_row, blk0, len, lane, cur);
       if (nblk > 1) block_rows(p, idx_row, blk0 + 1, len, lane, nxt);
       for (int n = gw; n < n_total; n += kGatherWarps) {
-        const int j = n / per_blk, c = n % per_blk, st = n % stages;
+        const int j = n / kDChunks, c = n % kDChunks;
         while (cur_blk < j) {                                 // advance to block j (at most a few steps)
 #pragma unroll
           for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
           ++cur_blk;
           if (cur_blk + 1 < nblk) block_rows(p, idx_row, blk0 + cur_blk + 1, len, lane, nxt);
         }
-        if (!warp_wait(&empty[st], ((n / stages) & 1) ^ 1, p.status, ab, false)) break;
+        if (!warp_wait(&S.s_empty[c], (j & 1) ^ 1, p.status, ab, false)) break;
+        if (c < kVChunks && j > 0 && !warp_wait(&S.xfer, (j - 1) & 1, p.status, ab, false)) break;
         const uint16_t* src[16];
         uint32_t dst[16], nb[16];
-        if (is_s) {
-          const uint32_t dst0 = smem_u32(S.s_ring[st]);
+        const uint32_t dst0 = smem_u32(S.s_ring[c]);
 #pragma unroll
-          for (int it = 0; it < 16; ++it) {
-            const int r = it * 4 + (lane >> 3);                // row within this CTA's 64
-            // entry rank*64 + r: register slot rank*2 + it/8, lane (it%8)*4 + lane/8
-            const int mine = rank ? cur[2 + (it >> 3)] : cur[it >> 3];
-            const int v = __shfl_sync(0xffffffffu, mine, (it & 7) * 4 + (lane >> 3));
-            src[it] = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + c * 64 + c16 * 8;
-            dst[it] = dst0 + r * 128 + ((c16 ^ (r & 7)) << 4);
-            nb[it] = v < 0 ? 0u : 16u;
-          }
-        } else {
-          const uint32_t dst0 = smem_u32(S.v_ring[st]);
-          int mine = cur[0];
-#pragma unroll
-          for (int u = 1; u < 4; ++u)
-            if ((c >> 1) == u) mine = cur[u];                  // register slot c/2 (warp-uniform)
-#pragma unroll
-          for (int it = 0; it < 16; ++it) {
-            const int pi = it * 4 + (lane >> 3);               // (row, group) pair 0..63
-            const int r = pi & 15, grp = pi >> 4;
-            const int d0 = (grp >> 1) * 256 + static_cast<int>(rank) * 128 + (grp & 1) * 64;
-            // entry c*16 + r of the block: register slot c/2, lane (c%2)*16 + r
-            const int v = __shfl_sync(0xffffffffu, mine, (c & 1) * 16 + r);
-            src[it] = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + d0 + c16 * 8;
-            dst[it] = dst0 + grp * 2048 + r * 128 + ((c16 ^ (r & 7)) << 4);
-            nb[it] = v < 0 ? 0u : 16u;
-          }
+        for (int it = 0; it < 16; ++it) {
+          const int r = it * 4 + (lane >> 3);                  // row within this CTA's 64
+          // entry rank*64 + r: register slot rank*2 + it/8, lane (it%8)*4 + lane/8
+          const int mine = rank ? cur[2 + (it >> 3)] : cur[it >> 3];
+          const int v = __shfl_sync(0xffffffffu, mine, (it & 7) * 4 + (lane >> 3));
+          src[it] = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + c * 64 + c16 * 8;
+          dst[it] = dst0 + r * 128 + ((c16 ^ (r & 7)) << 4);
+          nb[it] = v < 0 ? 0u : 16u;
         }
 #pragma unroll
         for (int it = 0; it < 16; ++it) cp_async16(dst[it], src[it], nb[it]);
-        cp_async_arrive_noinc(&loaded[st]);
+        cp_async_arrive_noinc(&S.s_loaded[c]);
       }
       cp_async_wait_all();
-    } else if (warp >= 13) {
-      // ================================================================ relays
-      // Warp 13 lane 0: this CTA's Q load (9 TMA boxes of 64 dims x 64 heads) and
-      // the S ring; warp 14 lane 0: the V ring.  Each forwards completed stages,
-      // in order, to the even CTA's barriers.  They wait with the suspending
-      // try_wait: a spinning test_wait poller competes with the gathers for the
-      // shared-memory pipe.  As in cp.async-fed tensor-core pipelines, the stage
-      // barrier (completed by the copies themselves) orders the data before the
-      // MMA that reads it, so no proxy fence is issued here.
-      if (lane == 0) {
-        const bool is_s = warp == 13;
-        if (is_s) {
-          mbar_arrive_expect_tx(&S.q_full, kDChunks * kHalf * 128);
-          for (int dc = 0; dc < kDChunks; ++dc)
-            tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
-          if (mbar_wait(&S.q_full, 0, p.status, ab)) pair_signal(rank, &S.q_ready, &S.mbox_q, true, 4);
-        }
-        const int n = nblk * (is_s ? kDChunks : kBlk / 16);
-        const int stages = is_s ? kSStages : kVStages;
-        uint64_t* loaded = is_s ? S.s_loaded : S.v_loaded;
-        uint64_t* full = is_s ? S.s_full : S.v_full;
-        uint32_t* mbox = is_s ? S.mbox_s : S.mbox_v;
-        for (int i = 0; i < n; ++i) {
-          const int st = i % stages;
-          if (!mbar_wait(&loaded[st], (i / stages) & 1, p.status, ab)) break;
-          pair_signal(rank, &full[st], &mbox[st], true, 4);
-        }
+    } else if (warp == 13 && lane == 0) {
+      // ================================================================ S relay
+      // This CTA's Q load (9 TMA boxes of 64 dims x 64 heads), then completed
+      // S-ring stages forwarded, in order, to the even CTA's barriers.  It waits
+      // with the suspending try_wait: a spinning test_wait poller competes with
+      // the gathers for the shared-memory pipe.  As in cp.async-fed tensor-core
+      // pipelines, the stage barrier (completed by the copies themselves) orders
+      // the data before the MMA that reads it.
+      mbar_arrive_expect_tx(&S.q_full, kDChunks * kHalf * 128);
+      for (int dc = 0; dc < kDChunks; ++dc)
+        tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
+      if (mbar_wait(&S.q_full, 0, p.status, ab)) pair_signal(rank, &S.q_ready, &S.mbox_q, true, 4);
+      for (int i = 0; i < nblk * kDChunks; ++i) {
+        const int c = i % kDChunks;
+        if (!mbar_wait(&S.s_loaded[c], (i / kDChunks) & 1, p.status, ab)) break;
+        pair_signal(rank, &S.s_full[c], &S.mbox_s[c], true, 4);
       }
+    } else if (warp == 14 && lane == 0) {
+      // ================================================================ V copier / relay
+      // The V operand is the first 512 dims of the rows already in the S rings,
+      // so it is never gathered from L2 twice: this CTA's rows (half `rank` of
+      // the block) are copied, chunk by chunk, from its S ring into the V
+      // buffers, its own dims groups into its own buffer and the peer's into the
+      // peer's (bulk shared-memory copies over the cluster).  V buffer dim group
+      // g of CTA r holds dims (g/2)*256 + r*128 + (g%2)*64, i.e. S chunk
+      // 4*(g/2) + 2r + g%2; every row is a 128-byte swizzled line in both layouts,
+      // so a tile copies verbatim.  Then the lane forwards both halves' arrival
+      // to the even CTA and reports the copies' completion to the source CTAs.
+      const uint32_t peer = rank ^ 1u;
+      for (int j = 0; j < nblk; ++j) {
+        bool ok = true;
+        for (int h = 0; h < 2; ++h) mbar_arrive_expect_tx(&S.v_loaded[h], 4 * kHalf * 128);
+        // the V buffers' half `rank` is free once the PV MMAs of block j-1 on it completed
+        if (j > 0) ok = mbar_wait(&S.v_empty[rank], (j - 1) & 1, p.status, ab);
+        for (int c = 0; c < kVChunks && ok; ++c) {
+          if (!mbar_wait(&S.s_loaded[c], j & 1, p.status, ab)) { ok = false; break; }
+          fence_proxy_async_smem();                          // cp.async writes -> bulk-copy reads
+          const uint32_t owner = static_cast<uint32_t>((c >> 1) & 1);   // CTA whose dims these are
+          const int g = (c >> 2) * 2 + (c & 1);
+          const uint32_t dst = smem_u32(&S.vbuf[g][static_cast<int>(rank) * kHalf * 128]);
+          const uint32_t bar = smem_u32(&S.v_loaded[rank]);
+          if (owner == rank) bulk_copy_s2c(dst, smem_u32(S.s_ring[c]), kHalf * 128, bar);
+          else bulk_copy_s2c(mapa(dst, peer), smem_u32(S.s_ring[c]), kHalf * 128, mapa(bar, peer));
+        }
+        if (!ok) break;
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(&S.v_loaded[h], j & 1, p.status, ab)) { ok = false; break; }
+          pair_signal(rank, &S.v_full[h], &S.mbox_v[h], true, 4);
+          // half h holds CTA h's rows: tell CTA h that these copies of its chunks landed
+          if (static_cast<uint32_t>(h) == rank) mbar_arrive(&S.xfer);
+          else mbar_arrive_cluster(&S.xfer, peer);
+        }
+        if (!ok) break;
+      }
+      // after an abort, copies already issued may still be landing: hold the CTA briefly
+      if (*ab)
+        for (int i = 0; i < 100; ++i) __nanosleep(1000);
     } else if (rank == 0 && lane == 0) {
-      // ================================================================ MMA issuer (even CTA)
+      // ================================================================ MMA issuers (even CTA)
+      // Warp 12 issues S = Q K^T block after block, warp 15 issues O += P V.  With
+      // one issuer for both, S of block j+2 queued behind PV of block j, which
+      // waits for that block's softmax and V rows: the S ring then stayed full of
+      // consumed-late chunks and the gathers stalled.  The tensor pipe executes
+      // both streams; they touch disjoint TMEM columns.
       // Waits use the CTA-scope try_wait, as 2-SM tensor-core pipelines do for the
       // leader's stage barriers: a cluster-scope acquire on every stage cost about
       // 0.35 us each and throttled MMA issue.
       const uint32_t id_s = instr_desc(1, 1, false, false, 128, kBlk);   // bf16 x bf16, M=128 pair, N=128
       const uint32_t id_pv = instr_desc(1, 1, false, true, 128, 256);    // B (V) MN-major, N=256
-      bool ok = mbar_wait(&S.q_ready, 0, p.status, ab);
+      bool ok = warp == 12 ? mbar_wait(&S.q_ready, 0, p.status, ab) : true;
       // Descriptors are built once; a step inside a tile adds to the 14-bit
       // start-address field (16-byte units).  Each ring holds exactly one block,
       // so chunk c of every block sits in slot c and is in its (block)-th phase.
-      static_assert(kSStages == kDChunks && kVStages == kBlk / 16, "one block per ring");
+      static_assert(kSStages == kDChunks, "one block per ring");
       const uint64_t qd0 = smem_desc_sw128(smem_u32(S.q[0]), 16, 1024);
       const uint64_t sd0 = smem_desc_sw128(smem_u32(S.s_ring[0]), 16, 1024);
       const uint64_t pd0 = smem_desc_sw128(smem_u32(S.p[0]), 16, 1024);
-      const uint64_t vd0 = smem_desc_sw128(smem_u32(S.v_ring[0]), 2048, 1024);
+      const uint64_t vd0 = smem_desc_sw128(smem_u32(S.vbuf[0]), kBlk * 128, 1024);
       auto issue_s = [&](int j) -> bool {
         const int sb = j & 1;
         if (!mbar_wait(&S.s_free[sb], ((j >> 1) & 1) ^ 1, p.status, ab)) return false;
@@ -500,27 +537,30 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
-          if (!mbar_wait(&S.v_full[kk], j & 1, p.status, ab)) return false;
-          tc_fence_after();
+          if ((kk & 3) == 0) {                               // rows 64h.. of the V buffers (h = kk / 4)
+            if (!mbar_wait(&S.v_full[kk >> 2], j & 1, p.status, ab)) return false;
+            tc_fence_after();
+          }
           const uint64_t pa = pd0 + static_cast<uint64_t>((kk >> 2) * (kHalf * 128 / 16) + (kk & 3) * 2);
 #pragma unroll
           for (int c = 0; c < 2; ++c)
-            umma_bf16_pair(tmem + kOCol + c * 128, pa, vd0 + static_cast<uint64_t>(kk * (4 * 16 * 128 / 16) + c * 256),
-                           id_pv, (j | kk) != 0 ? 1u : 0u);
-          umma_commit_pair(&S.v_empty[kk], 0x3);
+            umma_bf16_pair(tmem + kOCol + c * 128, pa,
+                           vd0 + static_cast<uint64_t>(kk * (16 * 128 / 16) + c * (2 * kBlk * 128 / 16)), id_pv,
+                           (j | kk) != 0 ? 1u : 0u);
+          if ((kk & 3) == 3) umma_commit_pair(&S.v_empty[kk >> 2], 0x3);
         }
         umma_commit_pair(&S.p_empty, 0x3);
         return true;
       };
       if (ok) {
-        for (int j = 0; j < nblk && ok; ++j) {
-          ok = issue_s(j);
-          if (ok && j >= 1) ok = issue_pv(j - 1);
+        if (warp == 12) {
+          for (int j = 0; j < nblk && ok; ++j) ok = issue_s(j);
+        } else {
+          for (int j = 0; j < nblk && ok; ++j) ok = issue_pv(j);
         }
-        if (ok) ok = issue_pv(nblk - 1);
       }
-      umma_commit_pair(&S.done, 0x1);                       // drain: every MMA of this pair completed
-      mbar_wait(&S.done, 0, p.status, nullptr);
+      umma_commit_pair(&S.done, 0x1);                       // drain: this issuer's MMAs completed
+      mbar_wait(&S.done, 0, p.status, nullptr);              // ... and the other issuer's
     }
   } else if (warp < 4) {
     // no selected row: output zeros, lse = -inf
