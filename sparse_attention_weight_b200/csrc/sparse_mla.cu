@@ -147,17 +147,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// Local row indices of block `blk` of query t's index row: r[s] = entry
-// blk*128 + 32*s + lane, or -1 when unused or out of range.
-__device__ __forceinline__ void block_rows(const MlaParams& p, const int32_t* idx_row, int blk, int len, int lane,
-                                           int (&r)[4]) {
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const int pos = blk * kBlk + 32 * s + lane;
-    const int v = pos < p.k ? __ldg(idx_row + pos) : -1;
-    r[s] = (v >= 0 && v < len) ? v : -1;
-  }
-}
+// Order in which the chunks of a block are gathered, forwarded and multiplied:
+// the RoPE chunk (dims 512..575) first, since its slot is free as soon as the
+// previous block's S MMA read it, then the value chunks 0..7, whose slots also
+// wait for their copies into the V buffers.
+__device__ __forceinline__ int chunk_at(int i) { return i == 0 ? kDChunks - 1 : i - 1; }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
 sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
@@ -182,7 +176,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
     mbar_init(&S.q_full, 1);
     mbar_init(&S.q_ready, 1);
     for (int i = 0; i < kSStages; ++i) {
-      mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], 32);
+      mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], kGatherWarps * 32);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], 1);
@@ -394,46 +388,48 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       }
     } else if (warp < 12) {
       // ================================================================ gathers
-      // Warps 4-11 fill the S ring: chunk n (dims 64c..64c+63 of this CTA's 64
-      // rows of block n / 9) is loaded entirely by warp n % 8 (16 copies of 16 B
-      // per lane, 8 lanes per 128-byte row segment) and signalled with one
-      // hardware-tracked arrive per lane.  A slot is refilled once the S MMA read
-      // it and, for value chunks, once its copies into the V buffers landed.
-      // Each warp keeps the local row indices of its current and next block in
-      // registers (lane l holds entries 32*s + l).
+      // Warps 4-11 fill the S ring together, chunk by chunk in chunk_at order:
+      // warp w loads rows 8w..8w+7 of this CTA's 64 (two 16-byte copies per lane
+      // per chunk, 8 lanes per 128-byte row segment) and every lane signals with
+      // one hardware-tracked arrive.  Issuing a chunk across all eight warps
+      // makes chunks land one after another, so the S MMAs and the V copies start
+      // on the first chunk while the rest are in flight (chunk-per-warp issue
+      // made a block's chunks land together, at the end of its burst).  A value
+      // chunk's slot is refilled once its copies of the previous block landed.
       const int gw = warp - 4;
-      const int n_total = nblk * kDChunks;
       const int c16 = lane & 7;
-      int cur[4], nxt[4];
-      int cur_blk = 0;
-      block_rows(p, idx_row, blk0, len, lane, cur);
-      if (nblk > 1) block_rows(p, idx_row, blk0 + 1, len, lane, nxt);
-      for (int n = gw; n < n_total; n += kGatherWarps) {
-        const int j = n / kDChunks, c = n % kDChunks;
-        while (cur_blk < j) {                                 // advance to block j (at most a few steps)
+      const int rsub = lane >> 3;
+      // local row indices of this lane's two rows (8gw + rsub, 8gw + 4 + rsub) of block b
+      auto rows_of = [&](int b, int (&rr)[2]) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) cur[u] = nxt[u];
-          ++cur_blk;
-          if (cur_blk + 1 < nblk) block_rows(p, idx_row, blk0 + cur_blk + 1, len, lane, nxt);
+        for (int i = 0; i < 2; ++i) {
+          const int e = b * kBlk + static_cast<int>(rank) * kHalf + 8 * gw + 4 * i + rsub;
+          const int v = e < p.k ? __ldg(idx_row + e) : -1;
+          rr[i] = (v >= 0 && v < len) ? v : -1;
         }
-        if (!warp_wait(&S.s_empty[c], (j & 1) ^ 1, p.status, ab, false)) break;
-        if (c < kVChunks && j > 0 && !warp_wait(&S.xfer, (j - 1) & 1, p.status, ab, false)) break;
-        const uint16_t* src[16];
-        uint32_t dst[16], nb[16];
-        const uint32_t dst0 = smem_u32(S.s_ring[c]);
+      };
+      int cur[2], nxt[2] = {-1, -1};
+      rows_of(blk0, cur);
+      for (int j = 0; j < nblk; ++j) {
+        if (j + 1 < nblk) rows_of(blk0 + j + 1, nxt);
+        bool ok = true;
+        for (int i = 0; i < kDChunks; ++i) {
+          const int c = chunk_at(i);
+          if (!warp_wait(&S.s_empty[c], (j & 1) ^ 1, p.status, ab, false)) { ok = false; break; }
+          if (i == 1 && j > 0 && !warp_wait(&S.xfer, (j - 1) & 1, p.status, ab, false)) { ok = false; break; }
+          const uint32_t dst0 = smem_u32(S.s_ring[c]);
 #pragma unroll
-        for (int it = 0; it < 16; ++it) {
-          const int r = it * 4 + (lane >> 3);                  // row within this CTA's 64
-          // entry rank*64 + r: register slot rank*2 + it/8, lane (it%8)*4 + lane/8
-          const int mine = rank ? cur[2 + (it >> 3)] : cur[it >> 3];
-          const int v = __shfl_sync(0xffffffffu, mine, (it & 7) * 4 + (lane >> 3));
-          src[it] = p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + c * 64 + c16 * 8;
-          dst[it] = dst0 + r * 128 + ((c16 ^ (r & 7)) << 4);
-          nb[it] = v < 0 ? 0u : 16u;
+          for (int h = 0; h < 2; ++h) {
+            const int r = 8 * gw + 4 * h + rsub;               // row within this CTA's 64
+            const int v = cur[h];
+            cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4),
+                       p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + c * 64 + c16 * 8, v < 0 ? 0u : 16u);
+          }
+          cp_async_arrive_noinc(&S.s_loaded[c]);
         }
-#pragma unroll
-        for (int it = 0; it < 16; ++it) cp_async16(dst[it], src[it], nb[it]);
-        cp_async_arrive_noinc(&S.s_loaded[c]);
+        if (!ok) break;
+        cur[0] = nxt[0];
+        cur[1] = nxt[1];
       }
       cp_async_wait_all();
     } else if (warp == 13 && lane == 0) {
@@ -449,7 +445,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
       if (mbar_wait(&S.q_full, 0, p.status, ab)) pair_signal(rank, &S.q_ready, &S.mbox_q, true, 4);
       for (int i = 0; i < nblk * kDChunks; ++i) {
-        const int c = i % kDChunks;
+        const int c = chunk_at(i % kDChunks);
         if (!mbar_wait(&S.s_loaded[c], (i / kDChunks) & 1, p.status, ab)) break;
         pair_signal(rank, &S.s_full[c], &S.mbox_s[c], true, 4);
       }
@@ -520,13 +516,14 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         tc_fence_after();
         const uint32_t d = tmem + kSCol + sb * 64;
 #pragma unroll
-        for (int dc = 0; dc < kDChunks; ++dc) {
+        for (int ci = 0; ci < kDChunks; ++ci) {
+          const int dc = chunk_at(ci);
           if (!mbar_wait(&S.s_full[dc], j & 1, p.status, ab)) return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             umma_bf16_pair(d, qd0 + static_cast<uint64_t>(dc * (kHalf * 128 / 16) + kk * 2),
-                           sd0 + static_cast<uint64_t>(dc * (kHalf * 128 / 16) + kk * 2), id_s, (dc | kk) != 0 ? 1u : 0u);
+                           sd0 + static_cast<uint64_t>(dc * (kHalf * 128 / 16) + kk * 2), id_s, (ci | kk) != 0 ? 1u : 0u);
           umma_commit_pair(&S.s_empty[dc], 0x3);
         }
         umma_commit_pair(&S.s_ready[sb], 0x3);
