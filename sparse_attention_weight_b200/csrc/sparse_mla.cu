@@ -77,7 +77,7 @@ struct MlaSmem {
   uint64_t mx_bar[2], l_bar;
   uint64_t done;
   // mailboxes of the peer CTA's asynchronous signals (contents unused)
-  uint32_t mbox_q, mbox_s[kSStages], mbox_v[2], mbox_sfree[2][4], mbox_pfull[4];
+  uint32_t mbox_q, mbox_s[kSStages], mbox_v[2], mbox_x, mbox_sfree[2][4], mbox_pfull[4];
   uint32_t tmem_base;
   int last_used[8];                          // per prologue warp: last usable entry, -1 if none
   int abort_flag;
@@ -181,7 +181,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], 1);
     }
-    mbar_init(&S.xfer, 2);
+    mbar_init(&S.xfer, 1);                      // own arrival (+4 tx bytes from the peer's report)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 4); mbar_init(&S.mx_bar[i], 128);
     }
@@ -481,8 +481,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
           if (!mbar_wait(&S.v_loaded[h], j & 1, p.status, ab)) { ok = false; break; }
           pair_signal(rank, &S.v_full[h], &S.mbox_v[h], true, 4);
           // half h holds CTA h's rows: tell CTA h that these copies of its chunks landed
-          if (static_cast<uint32_t>(h) == rank) mbar_arrive(&S.xfer);
-          else mbar_arrive_cluster(&S.xfer, peer);
+          // (own copies: this CTA's arrival, which also expects the peer's report;
+          // the peer's copies: an asynchronous 4-byte report, no round trip)
+          if (static_cast<uint32_t>(h) == rank) mbar_arrive_expect_tx(&S.xfer, 4);
+          else st_async_signal(&S.mbox_x, &S.xfer, peer, 1u);
         }
         if (!ok) break;
       }
