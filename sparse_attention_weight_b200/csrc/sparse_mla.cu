@@ -70,14 +70,15 @@ struct MlaSmem {
   uint32_t valid[2048 / 32];                 // bit e: entry e of the index row is a usable row
   uint64_t q_full, q_ready;
   uint64_t s_full[kSStages], s_empty[kSStages], s_loaded[kSStages];
-  uint64_t v_full[2], v_empty[2], v_loaded[2];   // per half of the block's rows (= per CTA's rows)
-  uint64_t xfer;                             // this CTA's copies of a block into both V buffers landed
+  uint64_t v_full[2], v_empty[2];            // per half of the block's rows (= per CTA's rows)
+  uint64_t v_loaded[2][2];                   // tiles of half h, dim groups 2q and 2q+1, landed here
+  uint64_t xfer[2];                          // this CTA's copies of value chunks 4q..4q+3 landed in both CTAs
   uint64_t s_ready[2], s_free[2];
   uint64_t p_full, p_empty;
   uint64_t mx_bar[2], l_bar;
   uint64_t done;
   // mailboxes of the peer CTA's asynchronous signals (contents unused)
-  uint32_t mbox_q, mbox_s[kSStages], mbox_v[2], mbox_x, mbox_sfree[2][4], mbox_pfull[4];
+  uint32_t mbox_q, mbox_s[kSStages], mbox_v[2], mbox_x[2], mbox_sfree[2][4], mbox_pfull[4];
   uint32_t tmem_base;
   int last_used[8];                          // per prologue warp: last usable entry, -1 if none
   int abort_flag;
@@ -179,9 +180,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], kGatherWarps * 32);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], 1);
+      mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1);
+      mbar_init(&S.v_loaded[i][0], 1); mbar_init(&S.v_loaded[i][1], 1);
+      mbar_init(&S.xfer[i], 1);                 // own arrival (+4 tx bytes from the peer's report)
     }
-    mbar_init(&S.xfer, 1);                      // own arrival (+4 tx bytes from the peer's report)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 4); mbar_init(&S.mx_bar[i], 128);
     }
@@ -416,7 +418,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         for (int i = 0; i < kDChunks; ++i) {
           const int c = chunk_at(i);
           if (!warp_wait(&S.s_empty[c], (j & 1) ^ 1, p.status, ab, false)) { ok = false; break; }
-          if (i == 1 && j > 0 && !warp_wait(&S.xfer, (j - 1) & 1, p.status, ab, false)) { ok = false; break; }
+          // value chunks 4q..4q+3 (i = 4q+1..): their copies of block j-1 must have landed
+          if ((i == 1 || i == 5) && j > 0 && !warp_wait(&S.xfer[i >> 2], (j - 1) & 1, p.status, ab, false)) {
+            ok = false;
+            break;
+          }
           const uint32_t dst0 = smem_u32(S.s_ring[c]);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
@@ -460,33 +466,38 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       // 4*(g/2) + 2r + g%2; every row is a 128-byte swizzled line in both layouts,
       // so a tile copies verbatim.  Then the lane forwards both halves' arrival
       // to the even CTA and reports the copies' completion to the source CTAs.
+      // Value chunks go in two quarters (chunks 4q..4q+3 = dim groups 2q, 2q+1 of
+      // both CTAs): once a quarter's copies have landed in both CTAs its S slots
+      // are released, while the next quarter is still being copied.
       const uint32_t peer = rank ^ 1u;
       for (int j = 0; j < nblk; ++j) {
         bool ok = true;
-        for (int h = 0; h < 2; ++h) mbar_arrive_expect_tx(&S.v_loaded[h], 4 * kHalf * 128);
+        for (int h = 0; h < 2; ++h)
+          for (int q = 0; q < 2; ++q) mbar_arrive_expect_tx(&S.v_loaded[h][q], 2 * kHalf * 128);
         // the V buffers' half `rank` is free once the PV MMAs of block j-1 on it completed
         if (j > 0) ok = mbar_wait(&S.v_empty[rank], (j - 1) & 1, p.status, ab);
-        for (int c = 0; c < kVChunks && ok; ++c) {
-          if (!mbar_wait(&S.s_loaded[c], j & 1, p.status, ab)) { ok = false; break; }
-          fence_proxy_async_smem();                          // cp.async writes -> bulk-copy reads
-          const uint32_t owner = static_cast<uint32_t>((c >> 1) & 1);   // CTA whose dims these are
-          const int g = (c >> 2) * 2 + (c & 1);
-          const uint32_t dst = smem_u32(&S.vbuf[g][static_cast<int>(rank) * kHalf * 128]);
-          const uint32_t bar = smem_u32(&S.v_loaded[rank]);
-          if (owner == rank) bulk_copy_s2c(dst, smem_u32(S.s_ring[c]), kHalf * 128, bar);
-          else bulk_copy_s2c(mapa(dst, peer), smem_u32(S.s_ring[c]), kHalf * 128, mapa(bar, peer));
+        for (int q = 0; q < kVChunks / 4 && ok; ++q) {
+          for (int c = 4 * q; c < 4 * q + 4; ++c) {
+            if (!mbar_wait(&S.s_loaded[c], j & 1, p.status, ab)) { ok = false; break; }
+            fence_proxy_async_smem();                        // cp.async writes -> bulk-copy reads
+            const uint32_t owner = static_cast<uint32_t>((c >> 1) & 1);   // CTA whose dims these are
+            const int g = (c >> 2) * 2 + (c & 1);
+            const uint32_t dst = smem_u32(&S.vbuf[g][static_cast<int>(rank) * kHalf * 128]);
+            const uint32_t bar = smem_u32(&S.v_loaded[rank][q]);
+            if (owner == rank) bulk_copy_s2c(dst, smem_u32(S.s_ring[c]), kHalf * 128, bar);
+            else bulk_copy_s2c(mapa(dst, peer), smem_u32(S.s_ring[c]), kHalf * 128, mapa(bar, peer));
+          }
+          for (int h = 0; h < 2 && ok; ++h) {
+            if (!mbar_wait(&S.v_loaded[h][q], j & 1, p.status, ab)) { ok = false; break; }
+            // tiles of half h hold CTA h's rows: tell CTA h these copies of its chunks landed
+            // (own copies: this CTA's arrival, which also expects the peer's report;
+            // the peer's copies: an asynchronous 4-byte report, no round trip)
+            if (static_cast<uint32_t>(h) == rank) mbar_arrive_expect_tx(&S.xfer[q], 4);
+            else st_async_signal(&S.mbox_x[q], &S.xfer[q], peer, 1u);
+          }
         }
         if (!ok) break;
-        for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(&S.v_loaded[h], j & 1, p.status, ab)) { ok = false; break; }
-          pair_signal(rank, &S.v_full[h], &S.mbox_v[h], true, 4);
-          // half h holds CTA h's rows: tell CTA h that these copies of its chunks landed
-          // (own copies: this CTA's arrival, which also expects the peer's report;
-          // the peer's copies: an asynchronous 4-byte report, no round trip)
-          if (static_cast<uint32_t>(h) == rank) mbar_arrive_expect_tx(&S.xfer, 4);
-          else st_async_signal(&S.mbox_x, &S.xfer, peer, 1u);
-        }
-        if (!ok) break;
+        for (int h = 0; h < 2; ++h) pair_signal(rank, &S.v_full[h], &S.mbox_v[h], true, 4);
       }
       // after an abort, copies already issued may still be landing: hold the CTA briefly
       if (*ab)
