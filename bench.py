@@ -40,10 +40,10 @@ from sparse_attention_weight_b200.configs import WORKLOADS  # noqa: E402
 L2_FLUSH_BYTES = 512 << 20
 MLA_FLOP_PER_PAIR = 128 * (576 + 512) * 2       # per (query, selected row) at H = 128
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
-# (profiles/sparse_mla_prefill_L2304.md: 624.0 MB at 2304 queries), scaled by the
+# (profiles/sparse_mla_prefill_L2304.md: 620.7 MB at 2304 queries), scaled by the
 # number of queries (the traffic is the queries in and the outputs out; the cache
 # gathers hit L2).  None where no capture stands for the current kernel.
-MLA_TRAFFIC_BYTES_PER_QUERY = 624.0e6 / 2304
+MLA_TRAFFIC_BYTES_PER_QUERY = 620.7e6 / 2304
 IDX_FLOP_PER_PAIR = 64 * 128 * 2                # per (query, visible key) at H_I = 64
 
 
@@ -58,12 +58,25 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of the SM clock and throttle reasons during the timed region."""
+    """nvidia-smi samples (every 20 ms) of the SM clock and throttle reasons.
+
+    Started before the warm-up, so that sampling is running when the timed region
+    begins; mark_start()/mark_end() bracket the timed region, and summary() keeps
+    the samples taken inside it.  A region shorter than the sampling interval holds
+    no sample: then the samples within 100 ms of it are used and `window` says so.
+    """
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.lines: list[str] = []
+        self.lines: list[tuple[float, str]] = []
+        self.t0 = self.t1 = None
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
 
     def __enter__(self):
         q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
@@ -71,17 +84,20 @@ class ClockSampler:
              "clocks_event_reasons.sw_power_cap")
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "20"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            deadline = time.monotonic() + 3.0                # wait until sampling has started
+            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
     def __exit__(self, *a):
         if self.proc:
@@ -92,9 +108,16 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        t0 = self.t0 if self.t0 is not None else float("-inf")
+        t1 = self.t1 if self.t1 is not None else float("inf")
+        window = "timed region"
+        sel = [ln for t, ln in self.lines if t0 <= t <= t1]
+        if not sel:
+            window = "within 100 ms of the timed region"
+            sel = [ln for t, ln in self.lines if t0 - 0.1 <= t <= t1 + 0.1]
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in sel:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 7:
                 continue
@@ -107,7 +130,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "window": window}
 
 
 def _smi_index(local: int) -> int:
@@ -190,23 +213,25 @@ def run_ours(args, wl, rank, world, device):
         if ev:
             ev[3].record(stream)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    for ws in (ws_i, ws_t, ws_m):
-        flags = B.read_device_status(ws)
-        if flags:
-            raise RuntimeError(f"device status flags 0x{flags:x}")
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(_smi_index(device.index or 0)) as clk:
+    with ClockSampler(_smi_index(device.index or 0)) as clk:      # sampling from before the warm-up
+        for _ in range(args.warmup):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+        for ws in (ws_i, ws_t, ws_m):
+            flags = B.read_device_status(ws)
+            if flags:
+                raise RuntimeError(f"device status flags 0x{flags:x}")
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        clk.mark_start()
         for k in range(args.steps):
             flush.zero_()
             step(events[k])
         torch.cuda.synchronize()
+        clk.mark_end()
     if world > 1:
         torch.distributed.barrier()
     stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in events])   # ms
