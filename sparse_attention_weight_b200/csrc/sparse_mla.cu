@@ -70,7 +70,7 @@ struct MlaSmem {
   uint32_t valid[2048 / 32];                 // bit e: entry e of the index row is a usable row
   uint64_t q_full, q_ready;
   uint64_t s_full[kSStages], s_empty[kSStages], s_loaded[kSStages];
-  uint64_t v_full[2], v_empty[2];            // per half of the block's rows (= per CTA's rows)
+  uint64_t v_full[2], v_empty[2];            // per quarter q: V-buffer dim groups 2q, 2q+1 (all rows)
   uint64_t v_loaded[2][2];                   // tiles of half h, dim groups 2q and 2q+1, landed here
   uint64_t xfer[2];                          // this CTA's copies of value chunks 4q..4q+3 landed in both CTAs
   uint64_t s_ready[2], s_free[2];
@@ -474,9 +474,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         bool ok = true;
         for (int h = 0; h < 2; ++h)
           for (int q = 0; q < 2; ++q) mbar_arrive_expect_tx(&S.v_loaded[h][q], 2 * kHalf * 128);
-        // the V buffers' half `rank` is free once the PV MMAs of block j-1 on it completed
-        if (j > 0) ok = mbar_wait(&S.v_empty[rank], (j - 1) & 1, p.status, ab);
         for (int q = 0; q < kVChunks / 4 && ok; ++q) {
+          // quarter q of the V buffers is free once the PV MMAs of block j-1 on it completed
+          if (j > 0 && !mbar_wait(&S.v_empty[q], (j - 1) & 1, p.status, ab)) { ok = false; break; }
           for (int c = 4 * q; c < 4 * q + 4; ++c) {
             if (!mbar_wait(&S.s_loaded[c], j & 1, p.status, ab)) { ok = false; break; }
             fence_proxy_async_smem();                        // cp.async writes -> bulk-copy reads
@@ -495,9 +495,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
             if (static_cast<uint32_t>(h) == rank) mbar_arrive_expect_tx(&S.xfer[q], 4);
             else st_async_signal(&S.mbox_x[q], &S.xfer[q], peer, 1u);
           }
+          if (ok) pair_signal(rank, &S.v_full[q], &S.mbox_v[q], true, 4);   // quarter q landed here
         }
         if (!ok) break;
-        for (int h = 0; h < 2; ++h) pair_signal(rank, &S.v_full[h], &S.mbox_v[h], true, 4);
       }
       // after an abort, copies already issued may still be landing: hold the CTA briefly
       if (*ab)
@@ -545,19 +545,21 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       auto issue_pv = [&](int j) -> bool {
         if (!mbar_wait(&S.p_full, j & 1, p.status, ab)) return false;
         tc_fence_after();
+        // value dims quarter by quarter (c = V-buffer groups 2c, 2c+1): the
+        // quarter's tiles are released for the next block's copies as soon as its
+        // 8 MMAs completed, while the other quarter is still being multiplied
 #pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk) {
-          if ((kk & 3) == 0) {                               // rows 64h.. of the V buffers (h = kk / 4)
-            if (!mbar_wait(&S.v_full[kk >> 2], j & 1, p.status, ab)) return false;
-            tc_fence_after();
-          }
-          const uint64_t pa = pd0 + static_cast<uint64_t>((kk >> 2) * (kHalf * 128 / 16) + (kk & 3) * 2);
+        for (int c = 0; c < 2; ++c) {
+          if (!mbar_wait(&S.v_full[c], j & 1, p.status, ab)) return false;
+          tc_fence_after();
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+          for (int kk = 0; kk < kBlk / 16; ++kk) {
+            const uint64_t pa = pd0 + static_cast<uint64_t>((kk >> 2) * (kHalf * 128 / 16) + (kk & 3) * 2);
             umma_bf16_pair(tmem + kOCol + c * 128, pa,
                            vd0 + static_cast<uint64_t>(kk * (16 * 128 / 16) + c * (2 * kBlk * 128 / 16)), id_pv,
                            (j | kk) != 0 ? 1u : 0u);
-          if ((kk & 3) == 3) umma_commit_pair(&S.v_empty[kk >> 2], 0x3);
+          }
+          umma_commit_pair(&S.v_empty[c], 0x3);
         }
         umma_commit_pair(&S.p_empty, 0x3);
         return true;
