@@ -40,10 +40,10 @@ from sparse_attention_weight_b200.configs import WORKLOADS  # noqa: E402
 L2_FLUSH_BYTES = 512 << 20
 MLA_FLOP_PER_PAIR = 128 * (576 + 512) * 2       # per (query, selected row) at H = 128
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
-# (profiles/sparse_mla_prefill_L2304.md: 620.7 MB at 2304 queries), scaled by the
+# (profiles/sparse_mla_prefill_L2304.md: 621.1 MB at 2304 queries), scaled by the
 # number of queries (the traffic is the queries in and the outputs out; the cache
 # gathers hit L2).  None where no capture stands for the current kernel.
-MLA_TRAFFIC_BYTES_PER_QUERY = 620.7e6 / 2304
+MLA_TRAFFIC_BYTES_PER_QUERY = 621.1e6 / 2304
 IDX_FLOP_PER_PAIR = 64 * 128 * 2                # per (query, visible key) at H_I = 64
 
 
