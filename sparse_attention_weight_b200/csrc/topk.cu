@@ -136,39 +136,36 @@ __device__ void find_bin(const uint32_t* hist, int nbins, uint32_t kneed, uint32
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p, int cache_elems) {
-  extern __shared__ __align__(16) uint32_t tk_smem[];
-  uint32_t* hist = tk_smem;                 // 2048
-  uint32_t* scratch = hist + 2048;          // 32
-  uint32_t* sel = scratch + 32;             // [0] bin, [1] remaining
-  uint32_t* cache = sel + 32;               // cache_elems (16-byte aligned: offset 2112 words)
-
-  const int t = blockIdx.x;
+// n of query row t (visible keys), or -1 for an invalid query; rows with n <= k
+// (and invalid ones) are written here and the function returns -1 / 0 for them.
+__device__ __forceinline__ int row_length(const TopkParams& p, int t, int32_t* out) {
   const int k = p.k;
-  int32_t* out = p.idx + static_cast<int64_t>(t) * k;
-
   int n = -1;
-  {
-    const int seq = p.q_seq[t];
-    if (seq >= 0 && seq < p.num_seqs) {
-      const int len = p.kv_len[seq];
-      const int pos = p.q_pos[t];
-      if (len >= 0 && len <= p.max_kv_len && pos >= 0 && pos < len) n = pos + 1;
-    }
+  const int seq = p.q_seq[t];
+  if (seq >= 0 && seq < p.num_seqs) {
+    const int len = p.kv_len[seq];
+    const int pos = p.q_pos[t];
+    if (len >= 0 && len <= p.max_kv_len && pos >= 0 && pos < len) n = pos + 1;
   }
   if (n < 0) {
     if (threadIdx.x == 0) set_status(p.status, DSA_DEV_BAD_QUERY);
     for (int j = threadIdx.x; j < k; j += kThreads) out[j] = -1;
-    return;
+    return -1;
   }
   if (n <= k) {
     for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < n ? j : -1;
-    return;
+    return 0;
   }
+  return n;
+}
 
-  Ctx c{p.scores + static_cast<int64_t>(t) * p.ld, n <= cache_elems ? cache : nullptr, n};
+// Exact top-k of row c (n > k) by three histogram passes (11, 11, 10 key bits)
+// and one output pass over the row: from the shared-memory cache when c.cache
+// is set (the first pass fills it), from L2 otherwise.
+__device__ void select_streaming(const Ctx& c, int k, int32_t* out, uint32_t* hist, uint32_t* scratch,
+                                 uint32_t* sel) {
   const bool cached = c.cache != nullptr;
-
+  const int n = c.n;
   // pass 1: bits 31..21
   for (int b = threadIdx.x; b < 2048; b += kThreads) hist[b] = 0;
   __syncthreads();
@@ -235,11 +232,182 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p, int cache_
   }
 }
 
+__global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p, int cache_elems) {
+  extern __shared__ __align__(16) uint32_t tk_smem[];
+  uint32_t* hist = tk_smem;                 // 2048
+  uint32_t* scratch = hist + 2048;          // 32
+  uint32_t* sel = scratch + 32;             // [0] bin, [1] remaining
+  uint32_t* cache = sel + 32;               // cache_elems (16-byte aligned: offset 2112 words)
+  const int t = blockIdx.x;
+  int32_t* out = p.idx + static_cast<int64_t>(t) * p.k;
+  const int n = row_length(p, t, out);
+  if (n <= 0) return;
+  const Ctx c{p.scores + static_cast<int64_t>(t) * p.ld, n <= cache_elems ? cache : nullptr, n};
+  select_streaming(c, p.k, out, hist, scratch, sel);
+}
+
+// ---------------------------------------------------------------- long rows
+// Rows too long for the shared-memory cache.  Pass 1 histograms the top 13 key
+// bits over the row; pass 2 reads the row again and compacts, in index order,
+// every key whose top bits reach the selected bin (all keys above it are taken,
+// the bin's keys are candidates) into a shared-memory list.  The remaining 19
+// bits are resolved on the list (10 + 9 bits) and the output pass runs over the
+// list, so the row is read twice instead of four times.  A row whose list would
+// overflow (a bin holding more than kListCap - k keys, e.g. massive ties) falls
+// back to the streaming passes.  Used when the rows are few (see launch_topk).
+constexpr int kHiBits = 13;
+constexpr int kHiShift = 32 - kHiBits;    // 19
+constexpr int kListCap = 8192;
+
+// Histogram of bits [shift, shift+bits) over list keys whose bits above `fshift` equal `prefix`.
+__device__ void hist_list(const uint32_t* keys, int m, uint32_t* hist, int shift, int bits, int fshift,
+                          uint32_t prefix) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t mask = (1u << bits) - 1u;
+  for (int base = 0; base < m; base += kThreads) {
+    const int i = base + threadIdx.x;
+    const bool in = i < m && (keys[i < m ? i : 0] >> fshift) == prefix;
+    const uint32_t bin = in ? ((keys[i] >> shift) & mask) : 0xffffffffu;
+    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+    if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) topk_long_kernel(TopkParams p) {
+  extern __shared__ __align__(16) uint32_t tk_smem[];
+  uint32_t* hist = tk_smem;                           // 1 << kHiBits
+  uint32_t* scratch = hist + (1 << kHiBits);          // 32
+  uint32_t* sel = scratch + 32;                       // [0] bin, [1] remaining
+  uint32_t* lkey = sel + 32;                          // kListCap
+  int32_t* lidx = reinterpret_cast<int32_t*>(lkey + kListCap);   // kListCap
+  const int t = blockIdx.x;
+  const int k = p.k;
+  int32_t* out = p.idx + static_cast<int64_t>(t) * k;
+  const int n = row_length(p, t, out);
+  if (n <= 0) return;
+  const Ctx c{p.scores + static_cast<int64_t>(t) * p.ld, nullptr, n};
+
+  // pass 1: top 13 bits over the row
+  for (int b = threadIdx.x; b < (1 << kHiBits); b += kThreads) hist[b] = 0;
+  __syncthreads();
+  hist_pass(c, false, false, hist, kHiShift, kHiBits, 32, 0);
+  __syncthreads();
+  find_bin(hist, 1 << kHiBits, static_cast<uint32_t>(k), scratch, &sel[0], &sel[1]);
+  const uint32_t b1 = sel[0], r1 = sel[1];
+  const uint32_t m_total = (static_cast<uint32_t>(k) - r1) + hist[b1];   // keys at or above bin b1
+  __syncthreads();
+  if (m_total > static_cast<uint32_t>(kListCap)) {    // block-uniform: fall back to streaming
+    select_streaming(c, k, out, hist, scratch, sel);
+    return;
+  }
+
+  // pass 2: compact keys with top bits >= b1, in index order
+  uint32_t m = 0;
+  for (int base = 0; base < n; base += kStep) {
+    const int i = base + threadIdx.x * kPer;
+    uint32_t kk[kPer];
+    bool valid[kPer];
+    load_keys(c, i, false, false, kk, valid);
+    uint32_t cnt = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) cnt += (valid[u] && (kk[u] >> kHiShift) >= b1) ? 1u : 0u;
+    uint32_t total;
+    const uint32_t incl = block_scan(cnt, scratch, &total);
+    uint32_t pos = m + incl - cnt;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (valid[u] && (kk[u] >> kHiShift) >= b1) {
+        if (pos < static_cast<uint32_t>(kListCap)) {
+          lkey[pos] = kk[u];
+          lidx[pos] = i + u;
+        }
+        ++pos;
+      }
+    }
+    m += total;
+  }
+  __syncthreads();
+  const int mi = static_cast<int>(min(m, static_cast<uint32_t>(kListCap)));
+
+  // passes 3 and 4 on the list: bits 18..9, then 8..0
+  for (int b = threadIdx.x; b < 1024; b += kThreads) hist[b] = 0;
+  __syncthreads();
+  hist_list(lkey, mi, hist, 9, 10, kHiShift, b1);
+  __syncthreads();
+  find_bin(hist, 1024, r1, scratch, &sel[0], &sel[1]);
+  const uint32_t b2 = sel[0], r2 = sel[1];
+  __syncthreads();
+  const uint32_t pre2 = (b1 << 10) | b2;
+  for (int b = threadIdx.x; b < 512; b += kThreads) hist[b] = 0;
+  __syncthreads();
+  hist_list(lkey, mi, hist, 0, 9, 9, pre2);
+  __syncthreads();
+  find_bin(hist, 512, r2, scratch, &sel[0], &sel[1]);
+  const uint32_t tau = (pre2 << 9) | sel[0];
+  const uint32_t need = sel[1];             // keys equal to tau to take, lowest indices first
+  __syncthreads();
+
+  // output pass over the list (index order)
+  uint32_t gt_base = 0, eq_base = 0;
+  for (int base = 0; base < mi; base += kStep) {
+    const int i = base + threadIdx.x * kPer;
+    uint32_t kk[kPer];
+    bool valid[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      valid[u] = i + u < mi;
+      kk[u] = valid[u] ? lkey[i + u] : 0u;
+    }
+    uint32_t cgt = 0, ceq = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      cgt += (valid[u] && kk[u] > tau) ? 1u : 0u;
+      ceq += (valid[u] && kk[u] == tau) ? 1u : 0u;
+    }
+    const uint32_t packed = cgt | (ceq << 16);
+    uint32_t total;
+    const uint32_t incl = block_scan(packed, scratch, &total);
+    const uint32_t excl = incl - packed;
+    uint32_t gt_before = gt_base + (excl & 0xffffu);
+    uint32_t eq_before = eq_base + (excl >> 16);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (!valid[u]) continue;
+      if (kk[u] > tau) {
+        const uint32_t slot = gt_before + min(eq_before, need);
+        if (slot < static_cast<uint32_t>(k)) out[slot] = lidx[i + u];
+        ++gt_before;
+      } else if (kk[u] == tau) {
+        const uint32_t slot = gt_before + eq_before;
+        if (eq_before < need && slot < static_cast<uint32_t>(k)) out[slot] = lidx[i + u];
+        ++eq_before;
+      }
+    }
+    gt_base += total & 0xffffu;
+    eq_base += total >> 16;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   int cache_elems = ((p.max_kv_len + kStep - 1) / kStep) * kStep;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess)
+    sms = 148;
+  // Long rows.  With few rows (at most two per SM: decode) each CTA has an SM to
+  // itself and reading the row twice instead of four times wins; with many rows
+  // the streaming kernel, four CTAs per SM, keeps more loads in flight.
+  if (cache_elems > kCacheMax && T <= 2 * sms) {      // two reads and a candidate list
+    const size_t smem = ((1 << kHiBits) + 64 + 2 * kListCap) * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(topk_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    topk_long_kernel<<<T, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+  }
   if (cache_elems > kCacheMax) cache_elems = 0;       // long rows stream from L2
   const size_t smem = (2048 + 64) * sizeof(uint32_t) + static_cast<size_t>(cache_elems) * sizeof(uint32_t);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

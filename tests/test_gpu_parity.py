@@ -132,11 +132,20 @@ def test_topk_adversarial_rows(cuda_device):
 
 
 def test_topk_long_rows_from_l2(cuda_device):
+    """Rows longer than the shared-memory cache: two reads and a candidate list,
+    and the streaming fallback when the threshold's bin overflows the list."""
     rng = np.random.default_rng(12)
     rows = [rng.standard_normal(40000).astype(np.float32),
             np.round(rng.standard_normal(131072), 2).astype(np.float32),
-            rng.standard_normal(33000).astype(np.float32)]
+            rng.standard_normal(33000).astype(np.float32),
+            np.zeros(40000, np.float32),                                     # all tied: fallback
+            rng.integers(-3, 4, size=50000).astype(np.float32),              # 7 values: fallback
+            np.concatenate([np.full(3000, 2.0), rng.standard_normal(60000) - 10.0]).astype(np.float32),
+            rng.standard_normal(1500).astype(np.float32)]                    # n <= k in a long launch
     _topk_case(cuda_device, rows, 2048)
+    # many long rows (more than two per SM): the streaming kernel reads them from L2
+    many = [np.round(rng.standard_normal(int(n)), 3).astype(np.float32) for n in rng.integers(33000, 40000, 320)]
+    _topk_case(cuda_device, many, 2048)
 
 # ----------------------------------------------------------------------------- sparse MLA
 
