@@ -50,7 +50,7 @@ namespace dsa {
 namespace {
 
 constexpr int kMlaThreads = 512;
-constexpr int kGatherWarps = 8;         // S-ring gather warps; each warp loads whole chunks
+constexpr int kGatherWarps = 8;         // S-ring gather warps; each loads 8 rows of every chunk
 constexpr int kBlk = 128;             // selected rows per block (pair)
 constexpr int kHalf = 64;             // rows per CTA for the S operand; heads per CTA
 constexpr int kDChunks = DSA_D_QK / 64;   // 9 chunks of 64 dims
@@ -62,7 +62,7 @@ constexpr uint32_t kOCol = 128;       // TMEM columns [128,384): O (2 x 128)
 
 struct MlaSmem {
   uint8_t q[kDChunks][kHalf * 128];          // 72 KB  Q of this CTA's heads (K-major SW128)
-  uint8_t s_ring[kSStages][kHalf * 128];     // 64 KB  S operand chunks: 64 rows x 64 dims
+  uint8_t s_ring[kSStages][kHalf * 128];     // 72 KB  S operand chunks: 64 rows x 64 dims
   uint8_t vbuf[4][kBlk * 128];               // 64 KB  V operand: 4 dim groups x 128 rows (MN-major SW128)
   uint8_t p[2][kHalf * 128];                 // 16 KB  P: 64 heads x 128 rows (two K chunks)
   float xmax[2][128];
