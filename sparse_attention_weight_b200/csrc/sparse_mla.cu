@@ -351,36 +351,35 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         const float lse_v = lt > 0.f ? (m_ref + __log2f(lt)) * 0.69314718055994531f : -INFINITY;
         if (p.splits == 1) {
           uint16_t* orow = p.out + (static_cast<int64_t>(t) * H + (store ? h : 0)) * DSA_D_V;
-          // 32 TMEM columns (32 consecutive value dims) per load
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + kOCol + c * 32, o);
+          for (int c = 0; c < 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tmem + lane_addr + kOCol + c * 16, o);
             tmem_ld_wait();
-            const int d0 = (c >> 2) * 256 + half * 128 + (c & 3) * 32;
-            uint32_t pkd[16];
+            const int d0 = (c >> 3) * 256 + half * 128 + (c & 7) * 16;
+            uint32_t pkd[8];
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
+            for (int u = 0; u < 8; ++u)
               pkd[u] = pack_bf16(__uint_as_float(o[2 * u]) * inv, __uint_as_float(o[2 * u + 1]) * inv);
             if (store) {
               uint4* dst = reinterpret_cast<uint4*>(orow + d0);
-#pragma unroll
-              for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pkd[4 * u], pkd[4 * u + 1], pkd[4 * u + 2], pkd[4 * u + 3]);
+              dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+              dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
             }
           }
           if (store && half == 0 && p.lse) p.lse[static_cast<int64_t>(t) * H + h] = lse_v;
         } else {
           float* orow = p.part_o + ((static_cast<int64_t>(t) * p.splits + split) * H + (store ? h : 0)) * DSA_D_V;
 #pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + kOCol + c * 32, o);
+          for (int c = 0; c < 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tmem + lane_addr + kOCol + c * 16, o);
             tmem_ld_wait();
-            const int d0 = (c >> 2) * 256 + half * 128 + (c & 3) * 32;
+            const int d0 = (c >> 3) * 256 + half * 128 + (c & 7) * 16;
             if (store) {
               float4* dst = reinterpret_cast<float4*>(orow + d0);
 #pragma unroll
-              for (int u = 0; u < 8; ++u)
+              for (int u = 0; u < 4; ++u)
                 dst[u] = make_float4(__uint_as_float(o[4 * u]) * inv, __uint_as_float(o[4 * u + 1]) * inv,
                                      __uint_as_float(o[4 * u + 2]) * inv, __uint_as_float(o[4 * u + 3]) * inv);
             }
