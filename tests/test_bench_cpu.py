@@ -42,3 +42,12 @@ def test_whole_job_rate_counts_every_rank():
     # T units per rank per step, world ranks, ms per step (max over ranks)
     assert bench.whole_job_rate(8192, 1, 10.0) == 8192 / 0.010
     assert bench.whole_job_rate(8192, 4, 10.0) == 4 * 8192 / 0.010
+
+
+def test_oracle_timing_runs_rows_until_its_budget():
+    from sparse_attention_weight_b200.configs import WORKLOADS
+    wl = WORKLOADS["tiny_prefill"]
+    sample = bench._oracle_sample(wl, rows_max=4)
+    assert len(sample["rows"]) == 4
+    rows, secs = bench._time_oracle(wl, sample, 0.2)
+    assert rows >= 1 and secs >= 0.2
