@@ -6,7 +6,6 @@ ranks).  These tests run that host logic in two gloo processes."""
 from __future__ import annotations
 
 import os
-import socket
 
 import numpy as np
 import pytest
@@ -15,19 +14,11 @@ import torch.distributed as dist
 import torch.multiprocessing as mp
 
 
-def _free_port() -> int:
-    s = socket.socket()
-    s.bind(("127.0.0.1", 0))
-    port = s.getsockname()[1]
-    s.close()
-    return port
-
-
-def _worker(rank: int, world: int, port: int, results):
-    os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
+def _worker(rank: int, world: int, store_file: str, results):
     import datetime
-    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    # a file rendezvous: no port to race for
+    dist.init_process_group("gloo", init_method=f"file://{store_file}", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
     try:
         import bench
         from sparse_attention_weight_b200 import inputs
@@ -48,12 +39,13 @@ def _worker(rank: int, world: int, port: int, results):
         dist.destroy_process_group()
 
 
-def test_two_ranks_reduce_timing_and_draw_distinct_shards():
-    world, port = 2, _free_port()
+def test_two_ranks_reduce_timing_and_draw_distinct_shards(tmp_path):
+    world = 2
     ctx = mp.get_context("spawn")
     manager = ctx.Manager()
     results = manager.dict()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, results)) for r in range(world)]
+    store = str(tmp_path / "rendezvous")
+    procs = [ctx.Process(target=_worker, args=(r, world, store, results)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
