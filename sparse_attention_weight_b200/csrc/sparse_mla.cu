@@ -464,11 +464,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       // peer's (bulk shared-memory copies over the cluster).  V buffer dim group
       // g of CTA r holds dims (g/2)*256 + r*128 + (g%2)*64, i.e. S chunk
       // 4*(g/2) + 2r + g%2; every row is a 128-byte swizzled line in both layouts,
-      // so a tile copies verbatim.  Then the lane forwards both halves' arrival
-      // to the even CTA and reports the copies' completion to the source CTAs.
-      // Value chunks go in two quarters (chunks 4q..4q+3 = dim groups 2q, 2q+1 of
-      // both CTAs): once a quarter's copies have landed in both CTAs its S slots
-      // are released, while the next quarter is still being copied.
+      // so a tile copies verbatim.  Value chunks go in two quarters (chunks
+      // 4q..4q+3 = dim groups 2q, 2q+1 of both CTAs): once a quarter's tiles have
+      // landed here the lane reports it to the even CTA (v_full, for the PV MMAs)
+      // and to the CTAs whose rows they are (xfer: those S slots may be refilled),
+      // while the next quarter is still being copied.
       const uint32_t peer = rank ^ 1u;
       for (int j = 0; j < nblk; ++j) {
         bool ok = true;
