@@ -98,7 +98,9 @@ size_t dsa_workspace_size(int op, const dsa_batch *batch, int H_I, int H, int k,
  *   w      (device) fp32 [T, H_I] per-head weights (any scale is folded into w)
  *   scores (device) fp32 [T, ld]: scores[t*ld + s] = I[t,s] for s < n_t.
  *          Entries s >= n_t are not written.
- * Supported: H_I in {4, 8, 16, 32, 64}; ld >= max_kv_len, ld % 4 == 0;
+ * Supported: H_I in {4, 8, 12, ..., 64} (multiples of 4; a count that is not a
+ * power of two is padded to the next one inside the MMA, with zero weights);
+ * ld >= max_kv_len, ld % 4 == 0;
  * the address of every buffer 16-byte aligned.  FP8 products are accumulated
  * in fp32 by the tensor cores; the ReLU, per-head weighting and head sum run
  * in fp32.
@@ -164,6 +166,9 @@ dsa_status dsa_forward(const dsa_batch *batch, const uint8_t *q_idx, const uint8
  *     exits.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process: after cudaDeviceReset
+ *     (which discards the device's copy of the array) do not call this entry
+ *     point again in that process.
  *   - Every call on a device shares the array and leaves its contents behind;
  *     calls whose kernels overlap on the GPU (e.g. on two streams) race on it,
  *     so serialise them.
@@ -200,6 +205,11 @@ const char *dsa_status_string(dsa_status status);
 
 /* DSA_ABI_VERSION of the built library. */
 int dsa_abi_version(void);
+
+/* Number of CUDA kernels the library has launched in this process so far (all
+ * devices and threads; launches that failed are not counted).  Instrumentation:
+ * the difference across a region counts the library's kernels in it. */
+uint64_t dsa_launch_count(void);
 
 #ifdef __cplusplus
 }

@@ -25,7 +25,7 @@ OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD = 0, 1, 2, 3
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward",
            "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
-           "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout")
+           "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout", "dsa_launch_count")
 NOALLOC_MAX_Q = 16384
 
 
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_status_string.argtypes = [i32]
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_abi_version.restype = i32
+        L.dsa_launch_count.restype = ctypes.c_uint64
         for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward", "dsa_forward_ws_views",
                    "dsa_read_device_status", "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout"):
             getattr(L, fn).restype = i32
@@ -182,6 +183,11 @@ def forward_ws_views(batch: DeviceBatch, H_I: int, H: int, k: int, ws) -> tuple[
 def dsa_selftest_wait_timeout(ws, limit_us: int, stream=None):
     _check("dsa_selftest_wait_timeout", lib().dsa_selftest_wait_timeout(_ptr(ws), ws.numel(), limit_us,
                                                                         _stream(stream)))
+
+
+def launch_count() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().dsa_launch_count())
 
 
 def read_device_status(ws, stream=None) -> int:

@@ -1,5 +1,6 @@
 // C ABI of the DSA hot path (declared in include/dsa.h): argument checks,
 // workspace layout, TMA descriptors and launches on the caller's stream.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -7,6 +8,10 @@
 #include "dsa_internal.h"
 
 namespace dsa {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -60,19 +65,27 @@ bool batch_ok(const dsa_batch* b) {
   return true;
 }
 
-bool hi_ok(int H_I) { return H_I == 4 || H_I == 8 || H_I == 16 || H_I == 32 || H_I == 64; }
+bool hi_ok(int H_I) { return H_I >= 4 && H_I <= 64 && H_I % 4 == 0; }
+// Column stride of one query token in the indexer's MMA: H_I rounded up to a
+// power of two (the epilogue reads whole 32-column TMEM chunks per token).
+int hi_pad(int H_I) {
+  int p = 4;
+  while (p < H_I) p <<= 1;
+  return p;
+}
 bool h_ok(int H) { return H >= 8 && H <= 128 && H % 8 == 0; }
 bool k_ok(int k) { return k >= 1 && k <= 2048; }
 
 int64_t default_ld(const dsa_batch* b) { return (static_cast<int64_t>(b->max_kv_len) + 3) / 4 * 4; }
 
 // Query tokens per indexer group: a power of two covering the queries of one
-// sequence, with the MMA N = G * H_I in [16, 256].
+// sequence, with the MMA N = G * hi_pad(H_I) in [16, 256].
 int indexer_group(const dsa_batch* b, int H_I) {
+  const int hp = hi_pad(H_I);
   int want = b->max_q_per_seq > 0 ? b->max_q_per_seq : b->num_q;
   int g = 1;
-  while (g < want && g * H_I < 256) g <<= 1;
-  while (g * H_I < 16) g <<= 1;
+  while (g < want && g * hp < 256) g <<= 1;
+  while (g * hp < 16) g <<= 1;
   return g;
 }
 
@@ -136,9 +149,12 @@ dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* 
                        float* scores, int64_t ld, const WsLayout& L, cudaStream_t st) {
   if (b->num_q == 0) return DSA_OK;
   const int G = indexer_group(b, H_I);
+  const int hp = hi_pad(H_I);
   CUtensorMap tq, tk;
+  // one box per query group, or (H_I not a power of two) one box per token
   if (!make_map_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, q_idx, DSA_D_INDEX,
-                   static_cast<uint64_t>(b->num_q) * H_I, DSA_D_INDEX, static_cast<uint32_t>(G * H_I)))
+                   static_cast<uint64_t>(b->num_q) * H_I, DSA_D_INDEX,
+                   static_cast<uint32_t>(hp == H_I ? G * H_I : H_I)))
     return DSA_ERR_CUDA;
   if (!make_map_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k_idx, DSA_D_INDEX,
                    static_cast<uint64_t>(b->kv_rows > 0 ? b->kv_rows : 1), DSA_D_INDEX, 128))
@@ -162,8 +178,9 @@ dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* 
   p.q_nvis = plan + 5 * T + 2;         // T entries (plan has 6T + 2)
   p.status = L.status;
   p.G = G;
+  p.hi = H_I;
   p.max_kv_len = b->max_kv_len;
-  return cuda_status(launch_indexer(tq, tk, p, H_I, T, b->num_seqs, b->kv_rows, num_sms(), st));
+  return cuda_status(launch_indexer(tq, tk, p, hp, T, b->num_seqs, b->kv_rows, num_sms(), st));
 }
 
 dsa_status run_topk(const dsa_batch* b, const float* scores, int64_t ld, int k, int32_t* idx, const WsLayout& L,
@@ -330,13 +347,18 @@ const char* dsa_status_string(dsa_status s) {
 
 int dsa_abi_version(void) { return DSA_ABI_VERSION; }
 
+uint64_t dsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
 }  // extern "C"
 
 // ----------------------------------------------------------------------------
 // Indexer without a caller workspace: the plan and status word live in a
 // fixed device array of this file (sized for DSA_NOALLOC_MAX_Q queries).
 namespace {
-constexpr size_t kNoAllocBytes = kWsHeader + (6 * static_cast<size_t>(DSA_NOALLOC_MAX_Q) + 2) * sizeof(int32_t);
+// Header plus the indexer plan of DSA_NOALLOC_MAX_Q queries, padded exactly as
+// plan_bytes() pads it, so that a call at the limit fits.
+constexpr size_t kNoAllocBytes =
+    kWsHeader + ((6 * static_cast<size_t>(DSA_NOALLOC_MAX_Q) + 2) * sizeof(int32_t) + kAlign - 1) / kAlign * kAlign;
 }  // namespace
 
 // In host code this name stands for the array, not for a device address; the

@@ -25,7 +25,8 @@ struct IndexerParams {
   int32_t* ngroups;          // [1]
   int32_t* q_nvis;           // [T] visible keys per query, -1 = invalid query
   uint32_t* status;
-  int G;                     // query tokens per group (N = G * H_I)
+  int G;                     // query tokens per group (N = G * padded H_I)
+  int hi;                    // H_I, heads per query token (a multiple of 4, <= 64)
   int max_kv_len;
 };
 
@@ -65,9 +66,12 @@ struct MlaParams {
   uint32_t* status;
 };
 
+// Counts kernel launches made by the library (dsa_launch_count).
+void count_launches(int n);
+
 size_t indexer_smem_bytes();
 size_t mla_smem_bytes();
-cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int H_I,
+cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int hi_pad,
                            int T, int B, int64_t kv_rows, int num_sms, cudaStream_t stream);
 cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream);
 cudaError_t launch_sparse_mla(const MlaParams& p, const CUtensorMap& tm_q, cudaStream_t stream);

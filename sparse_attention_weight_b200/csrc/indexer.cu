@@ -71,6 +71,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int i0 = min(total, static_cast<int>(blockIdx.x) * per);
   const int i1 = min(total, i0 + per);
   const int N = p.G * HI;
+  const int hi = p.hi;                  // real heads per token (HI = its padded column stride)
   volatile int* abort_flag = &S.abort_flag;
 
   if (threadIdx.x == 0) {
@@ -83,6 +84,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     fence_mbar_init();
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
+  }
+  if (hi != HI) {
+    // Tokens are loaded one by one at a stride of HI rows: the HI - hi padding
+    // rows of each token stay zero (they meet zero weights in the epilogue).
+    for (int i = threadIdx.x; i < kQBytes / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(S.q)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
   }
   if (warp == 1) tmem_alloc(&S.tmem_base, 512);
   tc_fence_before();
@@ -108,8 +116,13 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               if (!mbar_wait(&S.q_empty, qe_par, p.status, abort_flag)) break;
               qe_par ^= 1;
             }
-            mbar_arrive_expect_tx(&S.q_full, N * DSA_D_INDEX);
-            tma_load_2d(S.q, &tm_q, &S.q_full, 0, p.group_q0[g] * HI);
+            mbar_arrive_expect_tx(&S.q_full, p.G * hi * DSA_D_INDEX);
+            if (hi == HI) {
+              tma_load_2d(S.q, &tm_q, &S.q_full, 0, p.group_q0[g] * HI);
+            } else {
+              for (int u = 0; u < p.G; ++u)     // box = one token's hi rows
+                tma_load_2d(S.q + u * HI * DSA_D_INDEX, &tm_q, &S.q_full, 0, (p.group_q0[g] + u) * hi);
+            }
             ++q_loads;
             prev_g = g;
           }
@@ -183,7 +196,10 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           __syncwarp();
           q0 = p.group_q0[g];
           cnt = p.group_cnt[g];
-          for (int j = lane; j < cnt * HI; j += 32) sw[j] = p.w[static_cast<int64_t>(q0) * HI + j];
+          for (int j = lane; j < cnt * HI; j += 32) {
+            const int tok = j / HI, h = j - tok * HI;
+            sw[j] = h < hi ? p.w[static_cast<int64_t>(q0 + tok) * hi + h] : 0.f;
+          }
           for (int j = lane; j < cnt; j += 32) snv[j] = max(0, p.q_nvis[q0 + j]);
           __syncwarp();
           prev_g = g;
@@ -380,20 +396,24 @@ __global__ void __launch_bounds__(kPlanThreads) indexer_plan_kernel(IndexerParam
 
 size_t indexer_smem_bytes() { return sizeof(IdxSmem) + 1024; }
 
-cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int H_I,
+// hi_pad: the token column stride (a power of two, 4..64); p.hi <= hi_pad is H_I.
+cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int hi_pad,
                            int T, int B, int64_t kv_rows, int num_sms, cudaStream_t stream) {
   indexer_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p, T, B, kv_rows);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  count_launches(1);
   const size_t smem = indexer_smem_bytes();
   auto launch = [&](auto kern) -> cudaError_t {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     kern<<<num_sms, kIdxThreads, smem, stream>>>(tm_q, tm_k, p);
-    return cudaGetLastError();
+    err = cudaGetLastError();
+    if (err == cudaSuccess) count_launches(1);
+    return err;
   };
-  switch (H_I) {
+  switch (hi_pad) {
     case 4: return launch(indexer_kernel<4>);
     case 8: return launch(indexer_kernel<8>);
     case 16: return launch(indexer_kernel<16>);

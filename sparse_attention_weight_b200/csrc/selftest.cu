@@ -1,6 +1,7 @@
 // Self-test of the bounded in-kernel waits: a barrier that nothing completes
 // must make the waiting kernel give up, flag DSA_DEV_TIMEOUT and return.
 #include "dsa_common.cuh"
+#include "dsa_internal.h"
 
 namespace dsa {
 namespace {
@@ -23,5 +24,7 @@ extern "C" dsa_status dsa_selftest_wait_timeout(void* ws, size_t ws_bytes, uint3
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
   dsa::wait_timeout_kernel<<<1, 32, 0, st>>>(static_cast<uint32_t*>(ws), static_cast<uint64_t>(limit_us) * 1000ull);
-  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  dsa::count_launches(1);
+  return DSA_OK;
 }

@@ -289,14 +289,17 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         // a head with no usable entry so far has m_new = -inf and every x = -inf:
         // subtract 0 instead, so that each p is 2^-inf = 0 (never -inf - -inf)
         const float msub = m_new == -INFINITY ? 0.f : m_new;
+        // The denominator sums the bf16-rounded weights that the PV MMA multiplies
+        // V by, so the output is a convex combination of the selected rows.
         float psum = 0.f;
         uint32_t pk[32];
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const float p0 = ex2_approx(x[c] - msub);
           const float p1 = ex2_approx(x[c + 1] - msub);
-          psum += p0 + p1;
-          pk[c >> 1] = pack_bf16(p0, p1);
+          const uint32_t pp = pack_bf16(p0, p1);
+          psum += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
+          pk[c >> 1] = pp;
         }
         const float alpha = rescale ? ex2_approx(m_ref - m_new) : 1.f;   // m_ref = -inf -> 0
         l = l * alpha + psum;
@@ -643,9 +646,13 @@ cudaError_t launch_sparse_mla(const MlaParams& p, const CUtensorMap& tm_q, cudaS
   if (e != cudaSuccess) return e;
   sparse_mla_kernel<<<2 * p.T * p.splits, kMlaThreads, smem, stream>>>(tm_q, p);
   e = cudaGetLastError();
-  if (e != cudaSuccess || p.splits == 1) return e;
+  if (e != cudaSuccess) return e;
+  count_launches(1);
+  if (p.splits == 1) return e;
   mla_combine_kernel<<<dim3(p.T, p.H), 128, 0, stream>>>(p);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) count_launches(1);
+  return e;
 }
 
 }  // namespace dsa

@@ -406,7 +406,9 @@ cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     topk_long_kernel<<<T, kThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
   }
   if (cache_elems > kCacheMax) cache_elems = 0;       // long rows stream from L2
   const size_t smem = (2048 + 64) * sizeof(uint32_t) + static_cast<size_t>(cache_elems) * sizeof(uint32_t);
@@ -414,7 +416,9 @@ cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   topk_kernel<<<T, kThreads, smem, stream>>>(p, cache_elems);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e == cudaSuccess) count_launches(1);
+  return e;
 }
 
 }  // namespace dsa

@@ -67,7 +67,8 @@ def test_host_argument_checks(lib):
     assert lib.dsa_topk(None, p, 3000, 2048, p, ws, big, None) == 1
     assert lib.dsa_topk(ctypes.byref(b), p, 3000, 2048, p, None, big, None) == 1
     # unsupported shapes
-    assert lib.dsa_indexer_scores(ctypes.byref(b), p, p, p, 12, p, 3000, ws, big, None) == 2
+    for hi in (0, 2, 10, 66, 68):        # H_I must be a multiple of 4 in [4, 64]
+        assert lib.dsa_indexer_scores(ctypes.byref(b), p, p, p, hi, p, 3000, ws, big, None) == 2
     assert lib.dsa_indexer_scores(ctypes.byref(b), p, p, p, 64, p, 2999, ws, big, None) == 2   # ld % 4
     assert lib.dsa_indexer_scores(ctypes.byref(b), p, p, p, 64, p, 2000, ws, big, None) == 2   # ld < max_kv_len
     assert lib.dsa_topk(ctypes.byref(b), p, 3000, 4096, p, ws, big, None) == 2
