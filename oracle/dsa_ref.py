@@ -221,7 +221,7 @@ def dense_mla(q: np.ndarray, kv: np.ndarray, n_vis: np.ndarray, sm_scale: float,
 
 
 def forward(kv_offset, kv_len, q_seq, q_pos, q_idx, k_idx, w, q_bits, kv_bits,
-            k: int, sm_scale: float, queries=None, d_v: int = 512):
+            k: int, sm_scale: float, queries=None, d_v: int = 512, selections=None):
     """The whole path for the given queries: scores -> top-k -> sparse MLA.
 
     [一文讀懂] "四步工作流程", steps 2-4, applied per query against its own
@@ -229,9 +229,12 @@ def forward(kv_offset, kv_len, q_seq, q_pos, q_idx, k_idx, w, q_bits, kv_bits,
     fp32 weights, bf16 bit patterns) in the packed-cache layout: sequence b
     owns cache rows kv_offset[b] .. kv_offset[b] + kv_len[b] - 1.
 
-    ``queries`` selects a subset of query rows (default: all).  Returns a dict
-    with per-query lists: "scores" (float64 [n_t]), "idx" (int32 [k]),
-    and arrays "out" [n, H, d_v], "lse" [n, H].
+    ``queries`` selects a subset of query rows (default: all).  ``selections``
+    (optional, one index row per entry of ``queries``) replaces step 3's own
+    choice in step 4, so that the attention step can be evaluated on another
+    selection (the tests compare a GPU's attention on the GPU's own choice).
+    Returns a dict with per-query lists: "scores" (float64 [n_t]), "idx"
+    (int32 [k], the top-k choice), and arrays "out" [n, H, d_v], "lse" [n, H].
     """
     if queries is None:
         queries = np.arange(len(q_pos))
@@ -246,10 +249,15 @@ def forward(kv_offset, kv_len, q_seq, q_pos, q_idx, k_idx, w, q_bits, kv_bits,
         n = int(q_pos[t]) + 1
         keys = k_idx[off:off + n_b]
         s = indexer_scores(q_idx[t:t + 1], keys, w[t:t + 1], np.array([n]))[0]
-        sel = topk_select(s[None, :n].astype(np.float64), np.array([n]), k)[0]
-        o, l = sparse_mla(bf16_decode(q_bits[t:t + 1]), bf16_decode(kv_bits[off:off + n_b]),
-                          sel[None, :], sm_scale, d_v)
+        chosen = topk_select(s[None, :n].astype(np.float64), np.array([n]), k)[0]
+        sel = chosen if selections is None else np.asarray(selections[i])
+        # only the selected rows of the sequence are decoded: step 4 reads no other
+        valid = sel[sel >= 0].astype(np.int64)
+        rows = bf16_decode(kv_bits[off + valid])
+        local = np.full(sel.shape, -1, dtype=np.int64)
+        local[sel >= 0] = np.arange(valid.size)
+        o, l = sparse_mla(bf16_decode(q_bits[t:t + 1]), rows, local[None, :], sm_scale, d_v)
         out[i], lse[i] = o[0], l[0]
         scores_l.append(s[:n])
-        idx_l.append(sel)
+        idx_l.append(chosen)
     return {"scores": scores_l, "idx": idx_l, "out": out, "lse": lse}

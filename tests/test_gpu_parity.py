@@ -57,7 +57,13 @@ def _run_indexer(dev, wl, batch_host):
 @pytest.mark.parametrize("wl", [WORKLOADS["tiny_prefill"], MID_PREFILL, MID_DEC2, MID_DEC1,
                                 Workload("hi8", 23, "prefill", k=64, h_index=8, heads=8, seq_len=700),
                                 Workload("hi16", 24, "prefill", k=64, h_index=16, heads=8, seq_len=700),
-                                Workload("hi32", 25, "prefill", k=64, h_index=32, heads=8, seq_len=700)],
+                                Workload("hi32", 25, "prefill", k=64, h_index=32, heads=8, seq_len=700),
+                                Workload("hi12", 31, "prefill", k=64, h_index=12, heads=8, seq_len=700),
+                                Workload("hi48", 32, "prefill", k=64, h_index=48, heads=8, seq_len=700),
+                                Workload("hi20_dec", 33, "decode", k=64, h_index=20, heads=8, batch=3, ctx_min=300,
+                                         ctx_max=900, q_per_seq=3),
+                                Workload("hi60_dec", 34, "decode", k=64, h_index=60, heads=8, batch=4, ctx_min=100,
+                                         ctx_max=700, q_per_seq=1)],
                          ids=lambda w: w.name)
 def test_indexer_scores_match_oracle(cuda_device, wl):
     ins = inputs.make_inputs(wl)
@@ -65,11 +71,13 @@ def test_indexer_scores_match_oracle(cuda_device, wl):
     dev = H.to_device(ins, cuda_device)
     got = _run_indexer(dev, wl, batch)
     T = batch.num_q
-    rows = range(T) if T <= 1100 else _sample_rows(T, wl.k)
-    for t in rows:
-        I, A = H.indexer_ref_row(ins, t)
+    rows = list(range(T)) if T <= 1100 else _sample_rows(T, wl.k)
+    ref = H.oracle_rows(ins, wl, rows)
+    for i, t in enumerate(rows):
         n = int(batch.q_pos[t]) + 1
-        H.check_indexer_row(got[t, :n], I, A, f"{wl.name} row {t}")
+        I = ref["scores"][i]
+        assert I.shape == (n,)
+        H.check_indexer_row(got[t, :n], I, H.condition_scale(ins, t, n), f"{wl.name} row {t}")
         # nothing written beyond the visible keys
         assert np.isnan(got[t, n:]).all()
 
@@ -102,11 +110,8 @@ def _topk_case(cuda_device, rows, k):
 def test_topk_bit_exact_on_oracle_scores(cuda_device):
     wl = WORKLOADS["tiny_prefill"]
     ins = inputs.make_inputs(wl)
-    rows = []
-    for t in range(0, 1024, 7):
-        I, _ = H.indexer_ref_row(ins, t)
-        rows.append(I.astype(np.float32))
-    _topk_case(cuda_device, rows, wl.k)
+    ref = H.oracle_rows(ins, wl, range(0, 1024, 7))
+    _topk_case(cuda_device, [I.astype(np.float32) for I in ref["scores"]], wl.k)
 
 
 def test_topk_adversarial_rows(cuda_device):
@@ -151,15 +156,10 @@ def test_topk_long_rows_from_l2(cuda_device):
 
 
 def _mla_ref_rows(ins, idx_host, rows, wl):
-    batch = ins["batch"]
-    refs, lses = [], []
-    for t in rows:
-        off, n = H.seq_slice(batch, t)
-        o, l = oracle.sparse_mla(oracle.bf16_decode(ins["q"][t:t + 1]), oracle.bf16_decode(ins["kv"][off:off + n]),
-                                 idx_host[t:t + 1].astype(np.int64), wl.sm_scale)
-        refs.append(o[0])
-        lses.append(l[0])
-    return np.stack(refs), np.stack(lses)
+    """The oracle's attention for `rows` over the index rows idx_host[rows]."""
+    rows = list(rows)
+    ref = H.oracle_rows(ins, wl, rows, selections=idx_host[rows])
+    return ref["out"], ref["lse"]
 
 
 def _run_mla(dev, wl, idx_host, T):
@@ -173,13 +173,14 @@ def _run_mla(dev, wl, idx_host, T):
 
 
 def _oracle_idx(ins, wl, rows=None):
+    """Index rows [T, k] of the oracle's top-k choice for `rows` (all by default); -1 elsewhere."""
     batch = ins["batch"]
     T = batch.num_q
+    rows = list(range(T)) if rows is None else list(rows)
     idx = np.full((T, wl.k), -1, np.int32)
-    for t in (range(T) if rows is None else rows):
-        I, _ = H.indexer_ref_row(ins, t)
-        n = int(batch.q_pos[t]) + 1
-        idx[t] = oracle.topk_select(I[None, :n], np.array([n]), wl.k)[0]
+    ref = H.oracle_rows(ins, wl, rows)
+    for i, t in enumerate(rows):
+        idx[t] = ref["idx"][i]
     return idx
 
 
@@ -194,7 +195,7 @@ def test_sparse_mla_matches_oracle(cuda_device, wl):
     out_bits, lse = _run_mla(dev, wl, idx, T)
     ref, ref_lse = _mla_ref_rows(ins, idx, rows, wl)
     H.check_attention(out_bits[rows], ref, wl.name)
-    assert np.max(np.abs(lse[rows] - ref_lse)) <= H.LSE_ABS
+    H.check_lse(lse[rows], ref_lse, wl.name)
 
 
 def test_sparse_mla_holes_unsorted_and_empty_rows(cuda_device):
@@ -215,7 +216,7 @@ def test_sparse_mla_holes_unsorted_and_empty_rows(cuda_device):
     out_bits, lse = _run_mla(dev, wl, idx, T)
     ref, ref_lse = _mla_ref_rows(ins, idx, range(T - 1), wl)
     H.check_attention(out_bits[:T - 1], ref, "holes")
-    assert np.max(np.abs(lse[:T - 1] - ref_lse)) <= H.LSE_ABS
+    H.check_lse(lse[:T - 1], ref_lse, "holes")
     assert np.all(oracle.bf16_decode(out_bits[T - 1]) == 0) and np.all(np.isneginf(lse[T - 1]))
 
 
@@ -227,6 +228,7 @@ def test_sparse_mla_fewer_heads(cuda_device):
     out_bits, lse = _run_mla(H.to_device(ins, cuda_device), wl, idx, T)
     ref, ref_lse = _mla_ref_rows(ins, idx, range(T), wl)
     H.check_attention(out_bits, ref, "h40")
+    H.check_lse(lse, ref_lse, "h40")
 
 # ----------------------------------------------------------------------------- end to end
 
@@ -248,16 +250,20 @@ def _forward(dev, wl, batch_host):
 
 
 def check_forward_rows(ins, wl, rows, out_bits, lse, scores, idx):
+    """Scores, selection and attention of the GPU's forward on `rows` against the
+    oracle: attention is compared with the oracle's attention over the GPU's own
+    selection (identical to the oracle's result wherever the selections agree)."""
     batch = ins["batch"]
+    rows = list(rows)
+    ref = H.oracle_rows(ins, wl, rows, selections=idx[rows])
     mism = 0
-    for t in rows:
-        I, A = H.indexer_ref_row(ins, t)
+    for i, t in enumerate(rows):
         n = int(batch.q_pos[t]) + 1
-        H.check_indexer_row(scores[t, :n], I, A, f"{wl.name} row {t}")
-        mism += H.check_selection(idx[t], I, n, wl.k, f"{wl.name} row {t}")
-    ref, ref_lse = _mla_ref_rows(ins, idx, rows, wl)       # the oracle's attention on the GPU's selection
-    H.check_attention(out_bits[rows], ref, wl.name)
-    assert np.max(np.abs(lse[rows] - ref_lse)) <= H.LSE_ABS
+        I = ref["scores"][i]
+        H.check_indexer_row(scores[t, :n], I, H.condition_scale(ins, t, n), f"{wl.name} row {t}")
+        mism += H.check_selection(idx[t], ref["idx"][i], I, n, wl.k, f"{wl.name} row {t}")
+    H.check_attention(out_bits[rows], ref["out"], wl.name)
+    H.check_lse(lse[rows], ref["lse"], wl.name)
     return mism
 
 
@@ -272,19 +278,62 @@ def test_forward_end_to_end(cuda_device, wl):
     check_forward_rows(ins, wl, rows, out_bits, lse, scores, idx)
 
 
-@pytest.mark.parametrize("name", ["prefill_8k", "decode_b64", "decode_128k_mtp2", "chunked_64k"])
-def test_forward_full_size_sampled(cuda_device, name):
-    """The five workloads at full size (the chunked one: its last chunk), through
-    dsa_forward as the benchmark runs it, checked on sampled rows."""
+def _full_size_rows(batch, k):
+    """Rows checked at full size: every query when there are at most 64; otherwise
+    the first and last rows, the rows around n = k, 36 random rows with n > k
+    (real selection) and 6 with n <= k."""
+    T = batch.num_q
+    if T <= 64:
+        return list(range(T))
+    n = batch.q_pos.astype(np.int64) + 1
+    rows = {0, 1, T - 3, T - 2, T - 1}
+    rows |= set(int(x) for x in np.nonzero(np.abs(n - k) <= 1)[0])
+    rng = np.random.default_rng(123)
+    big, small = np.nonzero(n > k)[0], np.nonzero(n <= k)[0]
+    rows |= set(int(x) for x in rng.choice(big, size=min(big.size, 36), replace=False))
+    if small.size:
+        rows |= set(int(x) for x in rng.choice(small, size=min(small.size, 6), replace=False))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name,chunk", [("prefill_8k", None), ("decode_b64", None), ("decode_128k_mtp2", None),
+                                        ("chunked_64k", 0), ("chunked_64k", 7), ("chunked_64k", 15)])
+def test_forward_full_size_sampled(cuda_device, name, chunk):
+    """The workloads at full size through dsa_forward, as the benchmark runs them
+    (the chunked workload: its first, a middle and its last chunk against the
+    cache prefix), checked on sampled rows that include the last ones and at
+    least 32 rows that select among more than k keys."""
     wl = WORKLOADS[name]
-    chunk = (wl.seq_len // wl.chunk - 1) if wl.kind == "chunked_prefill" else None
     ins = inputs.make_inputs(wl, chunk_index=chunk)
     batch = ins["batch"]
     dev = H.to_device(ins, cuda_device)
     out_bits, lse, scores, idx = _forward(dev, wl, batch)
-    T = batch.num_q
-    rows = _sample_rows(T, wl.k) if T > 64 else list(range(0, T, max(1, T // 16)))
-    check_forward_rows(ins, wl, rows[:20], out_bits, lse, scores, idx)
+    rows = _full_size_rows(batch, wl.k)
+    n = batch.q_pos[rows].astype(np.int64) + 1
+    assert (n > wl.k).sum() >= min(32, int((batch.q_pos + 1 > wl.k).sum()))
+    assert batch.num_q - 1 in rows
+    check_forward_rows(ins, wl, rows, out_bits, lse, scores, idx)
+
+
+def test_chunked_prefill_equals_unchunked_on_the_gpu(cuda_device):
+    """A prefill of 4096 tokens run as four chunk calls against the growing cache
+    gives bit-identical scores, selections and outputs to the single call."""
+    full_wl = Workload("chunk_eq", 29, "prefill", k=2048, h_index=64, heads=128, seq_len=4096)
+    chk_wl = Workload("chunk_eq", 29, "chunked_prefill", k=2048, h_index=64, heads=128, seq_len=4096, chunk=1024)
+    ins = inputs.make_inputs(full_wl)
+    full = _forward(H.to_device(ins, cuda_device), full_wl, ins["batch"])
+    for c in range(4):
+        ci = inputs.make_inputs(chk_wl, chunk_index=c)
+        part = _forward(H.to_device(ci, cuda_device), chk_wl, ci["batch"])
+        r = slice(1024 * c, 1024 * c + 1024)
+        n_hi = 1024 * (c + 1)
+        assert np.array_equal(part[0], full[0][r]), f"chunk {c}: outputs differ"
+        assert np.array_equal(part[1], full[1][r]), f"chunk {c}: lse differs"
+        assert np.array_equal(part[3], full[3][r]), f"chunk {c}: selections differ"
+        for t in range(1024):
+            m = 1024 * c + t + 1
+            assert np.array_equal(part[2][t, :m].view(np.uint32), full[2][1024 * c + t, :m].view(np.uint32))
+        assert n_hi <= part[2].shape[1]
 
 # ----------------------------------------------------------------------------- device status
 

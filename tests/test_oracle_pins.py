@@ -323,3 +323,85 @@ def test_selection_is_a_pure_function_of_the_scores(k):
     a = oracle.topk_select(s, np.array([30, 10, 3]), k)
     b = oracle.topk_select(s.copy(), np.array([30, 10, 3]), k)
     assert np.array_equal(a, b)
+
+
+def _composition_from_library_routines(batch, ins, k, scale):
+    """The whole path for every query, written directly with PyTorch float64
+    routines and none of the oracle's functions: PyTorch's casts decode the
+    inputs, sequence b is sliced as rows kv_offset[b] .. + kv_len[b], query t
+    sees keys 0 .. q_pos[t] (inclusive), a stable descending sort picks the k
+    largest scores (ties to the lower index), and scaled_dot_product_attention
+    attends over the chosen rows through a boolean mask."""
+    qi = torch.from_numpy(ins["q_idx"]).view(torch.float8_e4m3fn).to(torch.float64)
+    ki = torch.from_numpy(ins["k_idx"]).view(torch.float8_e4m3fn).to(torch.float64)
+    w = torch.from_numpy(ins["w"]).to(torch.float64)
+    q = torch.from_numpy(ins["q"].view(np.int16)).view(torch.bfloat16).to(torch.float64)
+    kv = torch.from_numpy(ins["kv"].view(np.int16)).view(torch.bfloat16).to(torch.float64)
+    outs, lses, chosen = [], [], []
+    for t in range(batch.num_q):
+        b = int(batch.q_seq[t])
+        lo, hi = int(batch.kv_offset[b]), int(batch.kv_offset[b]) + int(batch.kv_len[b])
+        vis = int(batch.q_pos[t]) + 1
+        keys, rows = ki[lo:hi][:vis], kv[lo:hi][:vis]
+        score = (torch.relu(qi[t] @ keys.T) * w[t][:, None]).sum(dim=0)          # [vis]
+        order = torch.sort(score, descending=True, stable=True).indices
+        pick = torch.sort(order[:k]).values
+        mask = torch.zeros(vis, dtype=torch.bool)
+        mask[pick] = True
+        Hh = q.shape[1]
+        o = torch.nn.functional.scaled_dot_product_attention(
+            q[t][None, :, None, :], rows[None, None].expand(1, Hh, vis, 576),
+            rows[None, None, :, :512].expand(1, Hh, vis, 512), attn_mask=mask[None, None, None, :], scale=scale)
+        z = scale * (q[t] @ rows.T)
+        lses.append(torch.logsumexp(z.masked_fill(~mask[None, :], -float("inf")), dim=1).numpy())
+        outs.append(o[0, :, 0, :].numpy())
+        chosen.append(pick.numpy())
+    return np.stack(outs), np.stack(lses), chosen
+
+
+@pytest.mark.parametrize("wl", [
+    Workload("pin_fwd_dec", 94, "decode", k=12, h_index=4, heads=8, batch=4, ctx_min=6, ctx_max=40, q_per_seq=2),
+    Workload("pin_fwd_pre", 95, "prefill", k=10, h_index=8, heads=8, seq_len=33),
+    Workload("pin_fwd_chk", 96, "chunked_prefill", k=16, h_index=4, heads=8, seq_len=64, chunk=16),
+], ids=lambda w: w.name)
+def test_forward_equals_composition_of_library_routines(wl):
+    """Pins the oracle's composition (which cache rows a query sees, how many keys
+    are visible, per-sequence slicing of a packed cache) to an independent
+    restatement that calls none of the oracle's functions."""
+    ins = inputs.make_inputs(wl, chunk_index=2 if wl.kind == "chunked_prefill" else None)
+    batch = ins["batch"]
+    res = oracle.forward(batch.kv_offset, batch.kv_len, batch.q_seq, batch.q_pos, ins["q_idx"], ins["k_idx"],
+                         ins["w"], ins["q"], ins["kv"], wl.k, wl.sm_scale)
+    out, lse, chosen = _composition_from_library_routines(batch, ins, wl.k, wl.sm_scale)
+    assert np.max(np.abs(res["out"] - out)) < 1e-12
+    assert np.max(np.abs(res["lse"] - lse)) < 1e-12
+    for t in range(batch.num_q):
+        got = res["idx"][t]
+        assert np.array_equal(got[got >= 0], chosen[t])
+        assert len(res["scores"][t]) == int(batch.q_pos[t]) + 1
+    # the decode and prefill batches mix contexts below and above k, so both branches of step 3 run
+    n = batch.q_pos + 1
+    if wl.kind != "chunked_prefill":
+        assert (n <= wl.k).any() and (n > wl.k).any()
+
+
+def test_forward_evaluates_attention_on_a_given_selection():
+    wl = Workload("pin_fwd_sel", 97, "decode", k=8, h_index=4, heads=8, batch=2, ctx_min=20, ctx_max=30,
+                  q_per_seq=1)
+    ins = inputs.make_inputs(wl)
+    batch = ins["batch"]
+    rng = np.random.default_rng(12)
+    sel = np.full((2, 8), -1, np.int32)
+    for t in range(2):
+        n = int(batch.q_pos[t]) + 1
+        sel[t, [1, 4, 6]] = rng.choice(n, size=3, replace=False)
+    res = oracle.forward(batch.kv_offset, batch.kv_len, batch.q_seq, batch.q_pos, ins["q_idx"], ins["k_idx"],
+                         ins["w"], ins["q"], ins["kv"], wl.k, wl.sm_scale, selections=sel)
+    for t in range(2):
+        b = int(batch.q_seq[t])
+        off = int(batch.kv_offset[b])
+        q = oracle.bf16_decode(ins["q"][t])
+        rows = oracle.bf16_decode(ins["kv"][off + sel[t][sel[t] >= 0]])
+        mask = np.ones((1, rows.shape[0]), bool)
+        ref = _sdpa(q[None], rows, mask, wl.sm_scale)[0]
+        assert np.max(np.abs(res["out"][t] - ref)) < 1e-12
