@@ -1,18 +1,29 @@
-"""Benchmark of the DSA hot path on B200 (prefill tokens/s or decode queries/s).
+"""Benchmark of the DSA hot path on B200 (prefill tokens/s and decode queries/s).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+                    [--no-extra] [--no-e2e] [--no-cpu-baseline] [--seq-len L] [--chunk C]
 
 One step = the whole path (lightning indexer -> top-k -> sparse MLA) over one
-call of the workload (default: prefill_8k, one sequence of 8192 tokens, top-2048,
-H_I = 64, H = 128).  Inputs are seeded synthetic data resident in HBM; L2 is
-flushed (a 512 MB write) before every timed step and the flush is outside the
-timed events.  Per-stage CUDA events on the launching stream give each kernel's
-duration for the roofline line.  `e2e` repeats the step through dsa_forward
-from pinned host buffers, with the host->device copies of the step's inputs and
-the device->host copy of its output inside the timed region.
+batch of the workload.  The headline (default: prefill_8k, one sequence of 8192
+tokens, top-2048, H_I = 64, H = 128) is printed as the JSON line's own metric;
+the line also carries, under "workloads", the other full-size workloads timed
+the same way in the same run:
+  decode_b64        64 sequences, context U[4096, 32768], 1 query each;
+  decode_128k_mtp2  16 sequences at context 131072, 2 queries each;
+  chunked_64k       a 65536-token prefill run as 16 calls of 4096 queries
+                    against the growing cache (one step = all 16 calls).
+Inputs are seeded synthetic data resident in HBM when the timed region starts
+(the headline's drawn on the host by the seeded generator; the large
+sub-workloads drawn on the device by PyTorch's seeded Philox generator, same
+distributions and casts).  L2 is flushed (a 512 MB write) before every timed
+step, outside the timed events.  Per-stage CUDA events on the launching stream
+give each kernel's duration for the roofline figures.  `e2e` repeats the
+headline step through dsa_forward from pinned host buffers, with the
+host->device copies of the step's inputs and the device->host copy of its
+output inside the timed region.
 
 Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
-seeded inputs (independent shards, no collective on the data path); the timed
+seeded inputs (independent shards, no collective on the data path); each timed
 region is bracketed by barriers and the reported time is the max over ranks.
 
 --impl reference times the CPU oracle (numpy float64) on the host cores over a
@@ -21,8 +32,8 @@ bounded sample of rows of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -38,23 +49,39 @@ sys.path.insert(0, ROOT)
 from sparse_attention_weight_b200.configs import WORKLOADS  # noqa: E402
 
 L2_FLUSH_BYTES = 512 << 20
-MLA_FLOP_PER_PAIR = 128 * (576 + 512) * 2       # per (query, selected row) at H = 128
-# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
-# (profiles/sparse_mla_prefill_L2304.md: 621.1 MB at 2304 queries), scaled by the
-# number of queries (the traffic is the queries in and the outputs out; the cache
-# gathers hit L2).  None where no capture stands for the current kernel.
-MLA_TRAFFIC_BYTES_PER_QUERY = 621.1e6 / 2304
-IDX_FLOP_PER_PAIR = 64 * 128 * 2                # per (query, visible key) at H_I = 64
+D_QK, D_V, D_INDEX = 576, 512, 128
+# DRAM bytes (read + write) per query of the sparse-MLA kernel on 8K prefill, from
+# one ncu capture of the kernel as it stands (dram__bytes_read.sum +
+# dram__bytes_write.sum of `bench.py --seq-len 2304`, divided by its 2304
+# queries); None while no capture describes the current kernel.
+MLA_TRAFFIC_BYTES_PER_QUERY = None
+
+
+def mla_flop_per_pair(heads: int) -> int:
+    """bf16 flop of sparse MLA per (query, selected row): QK^T over 576 dims and PV over 512."""
+    return heads * (D_QK + D_V) * 2
+
+
+def idx_flop_per_pair(h_index: int) -> int:
+    """FP8 flop of the indexer per (query, visible key): H_I dot products of 128 dims."""
+    return h_index * D_INDEX * 2
 
 
 def _peaks():
+    """Roofline denominators: the measured copy bandwidth and bf16 GEMM rates of
+    this machine's B200s; FP8 = the measured bf16 burst rate times the nominal dense
+    FP8/bf16 ratio (4.5 / 2.25 PFLOP/s) unless an FP8 figure was measured."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             d = json.load(f)
-        return {"hbm": float(d["hbm_gbs"]), "bf16": float(d["bf16_tflops"]),
-                "bf16_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "src": "measured"}
+        bf16 = float(d["bf16_tflops"])
+        fp8 = float(d["fp8_tflops"]) if "fp8_tflops" in d else 2.0 * bf16
+        return {"hbm": float(d["hbm_gbs"]), "bf16": bf16,
+                "bf16_sustained": float(d.get("bf16_tflops_sustained", bf16)), "fp8": fp8,
+                "src": "measured", "fp8_src": "measured" if "fp8_tflops" in d else "2 x measured bf16 burst"}
     except Exception:
-        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "src": "fallback"}
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "fp8": 3180.0, "src": "fallback",
+                "fp8_src": "2 x fallback bf16"}
 
 
 class ClockSampler:
@@ -165,129 +192,259 @@ def rank_seed(rank: int) -> int:
     return rank
 
 
-def _algorithmic(wl, batch, idx_host=None):
-    """Algorithmic work of one step: indexer (query, visible key) pairs and
-    sparse-MLA (query, selected row) pairs; selected rows = min(n_t, k)."""
-    n = batch.q_pos.astype(np.int64) + 1
-    idx_pairs = int(n.sum())
-    sel_pairs = int(np.minimum(n, wl.k).sum())
-    return idx_pairs, sel_pairs
+def algorithmic_pairs(q_pos: np.ndarray, k: int) -> tuple[int, int]:
+    """(indexer (query, visible key) pairs, sparse-MLA (query, selected row) pairs)
+    of one call: n_t = q_pos + 1 visible keys, min(n_t, k) selected rows."""
+    n = np.asarray(q_pos, dtype=np.int64) + 1
+    return int(n.sum()), int(np.minimum(n, k).sum())
 
 
-def run_ours(args, wl, rank, world, device):
+# ----------------------------------------------------------------------------- one call of the path
+
+
+class Call:
+    """Device buffers and workspaces of one call (one batch) of the path."""
+
+    def __init__(self, wl, bh, dev: dict, device, out=None, lse=None, kv_rows=None, scores=None, idx=None):
+        import torch
+
+        from sparse_attention_weight_b200 import binding as B
+        self.B = B
+        self.wl, self.bh, self.dev = wl, bh, dev
+        self.db = B.DeviceBatch.from_host(bh, device, kv_rows=kv_rows)
+        T = bh.num_q
+        self.T = T
+        self.ld = (bh.max_kv_len + 3) // 4 * 4
+        # buffers shared between calls (the chunks of a prefill) are viewed at this call's shape
+        self.scores = (scores.view(-1)[:T * self.ld].view(T, self.ld) if scores is not None
+                       else torch.empty((T, self.ld), dtype=torch.float32, device=device))
+        self.idx = idx if idx is not None else torch.empty((T, wl.k), dtype=torch.int32, device=device)
+        self.out = out if out is not None else torch.empty((T, wl.heads, D_V), dtype=torch.int16, device=device)
+        self.lse = lse if lse is not None else torch.empty((T, wl.heads), dtype=torch.float32, device=device)
+        self.ws_i = B.workspace(B.OP_INDEXER, self.db, H_I=wl.h_index, ld=self.ld, device=device)
+        self.ws_t = B.workspace(B.OP_TOPK, self.db, k=wl.k, device=device)
+        self.ws_m = B.workspace(B.OP_SPARSE_MLA, self.db, H=wl.heads, k=wl.k, device=device)
+        self.idx_pairs, self.sel_pairs = algorithmic_pairs(bh.q_pos, wl.k)
+
+    def run(self, stream, ev=None, base=0):
+        """The three stages on `stream`; with `ev`, event ev[base + i] is recorded
+        before stage i and ev[base + 3] after the last."""
+        B, wl, d = self.B, self.wl, self.dev
+        if ev is not None:
+            ev[base].record(stream)
+        B.dsa_indexer_scores(self.db, d["q_idx"], d["k_idx"], d["w"], wl.h_index, self.scores, self.ld, self.ws_i,
+                             stream)
+        if ev is not None:
+            ev[base + 1].record(stream)
+        B.dsa_topk(self.db, self.scores, self.ld, wl.k, self.idx, self.ws_t, stream)
+        if ev is not None:
+            ev[base + 2].record(stream)
+        B.dsa_sparse_mla(self.db, d["q"], d["kv"], self.idx, wl.k, wl.heads, wl.sm_scale, self.out, self.lse,
+                         self.ws_m, stream)
+        if ev is not None:
+            ev[base + 3].record(stream)
+
+    def check_status(self):
+        for ws in (self.ws_i, self.ws_t, self.ws_m):
+            flags = self.B.read_device_status(ws)
+            if flags:
+                raise RuntimeError(f"device status flags 0x{flags:x}")
+
+
+def time_calls(calls: list, args, world: int, device, clk) -> dict:
+    """Warm-up, then args.steps timed steps of the calls run back to back (one step
+    = every call once), L2 flushed before each step; per-stage CUDA events."""
     import torch
 
     from sparse_attention_weight_b200 import binding as B
-    from sparse_attention_weight_b200 import inputs
-
-    chunk = (wl.seq_len // wl.chunk - 1) if wl.kind == "chunked_prefill" else None
-    ins = inputs.make_inputs(wl, seed=rank_seed(rank), chunk_index=chunk)
-    bh = ins["batch"]
-    T = bh.num_q
-    B.lib()
-    torch.cuda.set_device(device)
     stream = torch.cuda.current_stream()
-    db = B.DeviceBatch.from_host(bh, device)
-    d = {n: B.bits_to_tensor(ins[n], device) for n in ("q_idx", "k_idx", "w", "q", "kv")}
-    ld = (bh.max_kv_len + 3) // 4 * 4
-    scores = torch.empty((T, ld), dtype=torch.float32, device=device)
-    idx = torch.empty((T, wl.k), dtype=torch.int32, device=device)
-    out = torch.empty((T, wl.heads, 512), dtype=torch.int16, device=device)
-    lse = torch.empty((T, wl.heads), dtype=torch.float32, device=device)
-    ws_i = B.workspace(B.OP_INDEXER, db, H_I=wl.h_index, ld=ld, device=device)
-    ws_t = B.workspace(B.OP_TOPK, db, k=wl.k, device=device)
-    ws_m = B.workspace(B.OP_SPARSE_MLA, db, H=wl.heads, k=wl.k, device=device)
-    ws_f = B.workspace(B.OP_FORWARD, db, H_I=wl.h_index, H=wl.heads, k=wl.k, device=device)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-
-    def step(ev=None):
-        if ev:
-            ev[0].record(stream)
-        B.dsa_indexer_scores(db, d["q_idx"], d["k_idx"], d["w"], wl.h_index, scores, ld, ws_i, stream)
-        if ev:
-            ev[1].record(stream)
-        B.dsa_topk(db, scores, ld, wl.k, idx, ws_t, stream)
-        if ev:
-            ev[2].record(stream)
-        B.dsa_sparse_mla(db, d["q"], d["kv"], idx, wl.k, wl.heads, wl.sm_scale, out, lse, ws_m, stream)
-        if ev:
-            ev[3].record(stream)
-
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    with ClockSampler(_smi_index(device.index or 0)) as clk:      # sampling from before the warm-up
-        for _ in range(args.warmup):
-            flush.zero_()
-            step()
-        torch.cuda.synchronize()
-        for ws in (ws_i, ws_t, ws_m):
-            flags = B.read_device_status(ws)
-            if flags:
-                raise RuntimeError(f"device status flags 0x{flags:x}")
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize()
-        clk.mark_start()
-        for k in range(args.steps):
-            flush.zero_()
-            step(events[k])
-        torch.cuda.synchronize()
-        clk.mark_end()
+    n_ev = 4 * len(calls)
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        for c in calls:
+            c.run(stream)
+    torch.cuda.synchronize()
+    for c in calls:
+        c.check_status()
     if world > 1:
         torch.distributed.barrier()
-    stage = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(3)] for e in events])   # ms
-    total_ms = reduce_max(float(stage.sum()), device)
-    ms_per_step = total_ms / args.steps
-    idx_pairs, sel_pairs = _algorithmic(wl, bh)
+    torch.cuda.synchronize()
+    launches0 = B.launch_count()
+    clk.mark_start()
+    for s in range(args.steps):
+        flush.zero_()
+        for i, c in enumerate(calls):
+            c.run(stream, events[s], 4 * i)
+    torch.cuda.synchronize()
+    clk.mark_end()
+    launches = B.launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    # stage[s, i, j]: step s, call i, stage j (ms)
+    stage = np.array([[[events[s][4 * i + j].elapsed_time(events[s][4 * i + j + 1]) for j in range(3)]
+                       for i in range(len(calls))] for s in range(args.steps)])
+    step_ms = np.array([events[s][0].elapsed_time(events[s][n_ev - 1]) for s in range(args.steps)])
+    total_ms = reduce_max(float(step_ms.sum()), device)
+    for c in calls:
+        c.check_status()
+    return {"ms_per_step": total_ms / args.steps, "stage_ms": stage.sum(axis=1).mean(axis=0).tolist(),
+            "launches": launches, "launches_per_step": launches / args.steps}
 
-    # ---- end to end through dsa_forward with host buffers
-    e2e = None
-    if not args.no_e2e:
-        host = {n: torch.from_numpy(ins[n].view(np.int16) if ins[n].dtype == np.uint16 else ins[n]).pin_memory()
-                for n in ("q_idx", "k_idx", "w", "q", "kv")}
-        out_host = torch.empty((T, wl.heads, 512), dtype=torch.int16).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in host.values())
-        d2h = out_host.numel() * out_host.element_size()
 
-        def e2e_step():
-            for n in host:
-                d[n].copy_(host[n], non_blocking=True)
-            B.dsa_forward(db, d["q_idx"], d["k_idx"], d["w"], wl.h_index, d["q"], d["kv"], wl.heads, wl.k,
-                          wl.sm_scale, out, lse, ws_f, stream)
-            out_host.copy_(out, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        torch.cuda.synchronize()
-        n_e2e = max(3, min(args.steps, 10))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            torch.distributed.barrier()
-        e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = reduce_max(e0.elapsed_time(e1) / n_e2e, device)
-        e2e = {"value": whole_job_rate(T, world, e2e_ms), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": e2e_ms}
-    splits = 1
-    try:
-        from sparse_attention_weight_b200.binding import lib  # noqa: F401
-        pairs = (torch.cuda.get_device_properties(device).multi_processor_count // 2)
-        splits = max(1, min(pairs // max(T, 1), (wl.k + 127) // 128, 16))
-    except Exception:
-        pass
-    return {
-        "T": T, "ms_per_step": ms_per_step, "stage_ms": stage.mean(axis=0).tolist(),
-        "idx_pairs": idx_pairs, "sel_pairs": sel_pairs, "e2e": e2e, "clocks": clk.summary(),
-        "launches_per_step": 4 + (1 if splits > 1 else 0),
-        "k_idx_bytes": int(ins["k_idx"].nbytes), "n_vis": (bh.q_pos.astype(np.int64) + 1),
+def rates(wl, calls, res, peaks) -> dict:
+    """Per-stage rates of a timed workload against the roofline denominators."""
+    idx_ms, topk_ms, mla_ms = res["stage_ms"]
+    idx_pairs = sum(c.idx_pairs for c in calls)
+    sel_pairs = sum(c.sel_pairs for c in calls)
+    T = sum(c.T for c in calls)
+    decode = wl.kind == "decode"
+    idx_tflops = idx_pairs * idx_flop_per_pair(wl.h_index) / (idx_ms / 1e3) / 1e12
+    mla_tflops = sel_pairs * mla_flop_per_pair(wl.heads) / (mla_ms / 1e3) / 1e12
+    # sparse MLA bytes: gathered rows + queries in + outputs out + index lists
+    mla_bytes = sel_pairs * D_QK * 2 + T * wl.heads * (D_QK + D_V) * 2 + T * wl.k * 4
+    # indexer bytes: keys of every sequence once + queries + weights + scores written
+    k_rows = sum(int(c.bh.kv_len.sum()) for c in calls) if decode else sum(int(c.bh.max_kv_len) for c in calls)
+    idx_bytes = k_rows * D_INDEX + T * wl.h_index * (D_INDEX + 4) + idx_pairs * 4
+    topk_bytes = idx_pairs * 4 + T * wl.k * 4
+    out = {
+        "indexer": {"ms": idx_ms, "fp8_tflops": idx_tflops, "fp8_frac": idx_tflops / peaks["fp8"],
+                    "gbs": idx_bytes / (idx_ms / 1e3) / 1e9, "hbm_frac": idx_bytes / (idx_ms / 1e3) / 1e9 / peaks["hbm"]},
+        "topk": {"ms": topk_ms, "gbs": topk_bytes / (topk_ms / 1e3) / 1e9,
+                 "hbm_frac": topk_bytes / (topk_ms / 1e3) / 1e9 / peaks["hbm"]},
+        "sparse_mla": {"ms": mla_ms, "bf16_tflops": mla_tflops, "bf16_frac": mla_tflops / peaks["bf16"],
+                       "gbs": mla_bytes / (mla_ms / 1e3) / 1e9,
+                       "hbm_frac": mla_bytes / (mla_ms / 1e3) / 1e9 / peaks["hbm"]},
     }
+    if decode:
+        roof = {"bound": "hbm", "kernel": "sparse_mla (gather)", "achieved": out["sparse_mla"]["gbs"],
+                "peak": peaks["hbm"], "unit": "GB/s", "peak_source": peaks["src"] + " copy bandwidth",
+                "algorithmic_bytes_per_launch": mla_bytes / len(calls)}
+    else:
+        roof = {"bound": "tensor", "kernel": "sparse_mla", "achieved": mla_tflops, "peak": peaks["bf16"],
+                "unit": "TFLOP/s", "peak_source": peaks["src"] + " bf16 (burst)",
+                "algorithmic_flop_per_launch": sel_pairs * mla_flop_per_pair(wl.heads) / len(calls)}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    return {"stages": out, "roofline": roof}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+
+def host_call(wl, device, seed, chunk=None):
+    from sparse_attention_weight_b200 import binding as B
+    from sparse_attention_weight_b200 import inputs
+    ins = inputs.make_inputs(wl, seed=seed, chunk_index=chunk)
+    dev = {n: B.bits_to_tensor(ins[n], device) for n in ("q_idx", "k_idx", "w", "q", "kv")}
+    return Call(wl, ins["batch"], dev, device), ins
+
+
+def device_calls(wl, device, seed):
+    """The calls of one step of a workload with device-drawn inputs (a chunked
+    prefill: one call per chunk against the growing cache prefix)."""
+    import torch
+
+    from sparse_attention_weight_b200 import inputs
+    if wl.kind == "chunked_prefill":
+        nchunks = wl.seq_len // wl.chunk
+        full = inputs.make_batch(dataclasses.replace(wl, kind="prefill"), seed)
+        cache = inputs.device_cache_tensors(wl, full, device, seed)
+        out = torch.empty((wl.seq_len, wl.heads, D_V), dtype=torch.int16, device=device)
+        lse = torch.empty((wl.seq_len, wl.heads), dtype=torch.float32, device=device)
+        scores = torch.empty(wl.chunk * wl.seq_len, dtype=torch.float32, device=device)
+        idx = torch.empty((wl.chunk, wl.k), dtype=torch.int32, device=device)
+        calls = []
+        for c in range(nchunks):
+            bh = inputs.make_batch(wl, seed, c)
+            qt = inputs.device_query_tensors(wl, bh, device, seed, chunk=c)
+            r = slice(c * wl.chunk, (c + 1) * wl.chunk)
+            calls.append(Call(wl, bh, {**qt, **cache}, device, out=out[r], lse=lse[r], kv_rows=wl.seq_len,
+                              scores=scores, idx=idx))
+        return calls
+    bh = inputs.make_batch(wl, seed)
+    dev = {**inputs.device_query_tensors(wl, bh, device, seed), **inputs.device_cache_tensors(wl, bh, device, seed)}
+    return [Call(wl, bh, dev, device)]
+
+
+def sub_record(wl, args, rank, world, device, peaks) -> dict:
+    """A full-size workload timed like the headline, with device-drawn inputs."""
+    import torch
+    calls = device_calls(wl, device, rank_seed(rank))
+    sub_args = argparse.Namespace(**{**vars(args), "warmup": max(3, args.warmup)})
+    with ClockSampler(_smi_index(device.index or 0)) as clk:
+        res = time_calls(calls, sub_args, world, device, clk)
+    T = sum(c.T for c in calls)
+    decode = wl.kind == "decode"
+    r = rates(wl, calls, res, peaks)
+    rec = {"metric": "DSA decode queries/s" if decode else "DSA prefill tokens/s",
+           "value": whole_job_rate(T, world, res["ms_per_step"]), "unit": "queries/s" if decode else "tokens/s",
+           "ms_per_step": res["ms_per_step"], "steps": sub_args.steps, "warmup": sub_args.warmup,
+           "calls_per_step": len(calls), "queries_per_step": T, "config": config_of(wl, args),
+           "roofline": r["roofline"], "stages": r["stages"], "gpu_launches": res["launches"],
+           "clocks": clk.summary(), "data": "synthetic, drawn on the device (seeded Philox)"}
+    del calls
+    torch.cuda.empty_cache()
+    return rec
+
+
+def config_of(wl, args) -> dict:
+    decode = wl.kind == "decode"
+    return {"workload": wl.name, "k": wl.k, "h_index": wl.h_index, "heads": wl.heads, "d_qk": D_QK, "d_v": D_V,
+            "seq_len": wl.seq_len or None, "batch": wl.batch or None,
+            "ctx": [wl.ctx_min, wl.ctx_max] if decode else None, "q_per_seq": wl.q_per_seq or None,
+            "chunk": wl.chunk or None, "l2": "flushed before every timed step (512 MB write)",
+            "parallelism": f"dp{args.gpus}" if args.gpus > 1 else "single"}
+
+
+def e2e_headline(call, ins, args, world, device) -> dict:
+    """The headline step through dsa_forward from pinned host buffers: the host->device
+    copies of the step's inputs and the device->host copy of its output are inside
+    the timed region."""
+    import torch
+
+    from sparse_attention_weight_b200 import binding as B
+    wl, d = call.wl, call.dev
+    stream = torch.cuda.current_stream()
+    ws_f = B.workspace(B.OP_FORWARD, call.db, H_I=wl.h_index, H=wl.heads, k=wl.k, device=device)
+    host = {n: torch.from_numpy(ins[n].view(np.int16) if ins[n].dtype == np.uint16 else ins[n]).pin_memory()
+            for n in ("q_idx", "k_idx", "w", "q", "kv")}
+    out_host = torch.empty(tuple(call.out.shape), dtype=torch.int16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for n in host:
+            d[n].copy_(host[n], non_blocking=True)
+        B.dsa_forward(call.db, d["q_idx"], d["k_idx"], d["w"], wl.h_index, d["q"], d["kv"], wl.heads, wl.k,
+                      wl.sm_scale, call.out, call.lse, ws_f, stream)
+        out_host.copy_(call.out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    n_e2e = max(3, min(args.steps, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(e0.elapsed_time(e1) / n_e2e, device)
+    return {"value": whole_job_rate(call.T, world, e2e_ms), "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
+
+
+# ----------------------------------------------------------------------------- the CPU oracle
 
 
 def _oracle_sample(wl, rows_max: int = 64):
     """Inputs of a seeded sample of the workload's query rows for the oracle (built
-    outside any timed region): per row its query tensors, per sequence its cache."""
+    outside any timed region): rows drawn uniformly at random (seeded), so that the
+    mean time per row estimates the whole call's; per row its query tensors, per
+    sequence its cache."""
     from sparse_attention_weight_b200 import inputs
 
     chunk = (wl.seq_len // wl.chunk - 1) if wl.kind == "chunked_prefill" else None
@@ -327,6 +484,9 @@ def cpu_baseline(wl, budget_s: float = 12.0, rows_max: int = 64):
     return {"value": done / elapsed, "cores": len(os.sched_getaffinity(0)), "rows": done, "seconds": elapsed}
 
 
+# ----------------------------------------------------------------------------- main
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -334,16 +494,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="prefill_8k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-extra", action="store_true", help="time only the headline workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override the prefill length (smaller cases for profiler captures)")
+    ap.add_argument("--chunk", type=int, default=-1,
+                    help="chunked workload: time only this chunk's call (default: all chunks)")
     args = ap.parse_args()
     wl = WORKLOADS[args.config]
     if args.seq_len:
         if wl.kind != "prefill":
             ap.error("--seq-len applies to prefill workloads")
-        import dataclasses
         wl = dataclasses.replace(wl, name=f"{wl.name}@L={args.seq_len}", seq_len=args.seq_len)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -351,11 +513,7 @@ def main():
     decode = wl.kind == "decode"
     metric = "DSA decode queries/s" if decode else "DSA prefill tokens/s"
     unit = "queries/s" if decode else "tokens/s"
-    config = {"workload": wl.name, "k": wl.k, "h_index": wl.h_index, "heads": wl.heads,
-              "d_qk": 576, "d_v": 512, "seq_len": wl.seq_len or None, "batch": wl.batch or None,
-              "ctx": [wl.ctx_min, wl.ctx_max] if decode else None, "q_per_seq": wl.q_per_seq or None,
-              "chunk": wl.chunk or None, "l2": "flushed before every timed step (512 MB write)",
-              "parallelism": f"dp{args.gpus}" if args.gpus > 1 else "single"}
+    config = config_of(wl, args)
 
     if args.impl == "reference":
         if rank != 0:
@@ -378,8 +536,8 @@ def main():
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": config,
                 "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
-                                 "sample": f"each step: seeded query rows of {wl.name} in turn for "
-                                           f"{per_step:.1f} s of oracle time, full path per row (numpy "
+                                 "sample": f"each step: seeded uniformly random query rows of {wl.name} in turn "
+                                           f"for {per_step:.1f} s of oracle time, full path per row (numpy "
                                            f"float64); {rows} rows in {secs:.1f} s over {args.steps} steps"},
                 "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
@@ -389,45 +547,59 @@ def main():
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     device = torch.device("cuda", local)
-    res = run_ours(args, wl, rank, world, device)
+    torch.cuda.set_device(device)
+    from sparse_attention_weight_b200 import binding as B
+    B.lib()
     peaks = _peaks()
-    T = res["T"]
-    value = whole_job_rate(T, world, res["ms_per_step"])
-    st = res["stage_ms"]
-    mla_ms, idx_ms, topk_ms = st[2], st[0], st[1]
-    mla_tflops = res["sel_pairs"] * MLA_FLOP_PER_PAIR * wl.heads / 128 / (mla_ms / 1e3) / 1e12
-    if decode:
-        # decode: the gather-bound kernel, against HBM
-        gather = res["sel_pairs"] * 1152 + T * wl.heads * (576 + 512) * 2
-        roof = {"bound": "hbm", "kernel": "sparse_mla", "achieved": gather / (mla_ms / 1e3) / 1e9,
-                "peak": peaks["hbm"], "unit": "GB/s"}
+
+    # ---- headline
+    ins = None
+    if wl.kind == "chunked_prefill" and args.chunk < 0:
+        calls = device_calls(wl, device, rank_seed(rank))
+        data = "synthetic, drawn on the device (seeded Philox)"
     else:
-        roof = {"bound": "tensor", "kernel": "sparse_mla", "achieved": mla_tflops, "peak": peaks["bf16"],
-                "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["peak_source"] = peaks["src"] + (" (burst)" if roof["unit"] == "TFLOP/s" else "")
-    roof["traffic"] = (MLA_TRAFFIC_BYTES_PER_QUERY * T) if wl.kind == "prefill" else None
-    idx_tflops = res["idx_pairs"] * IDX_FLOP_PER_PAIR * wl.h_index / 64 / (idx_ms / 1e3) / 1e12
+        call, ins = host_call(wl, device, rank_seed(rank), args.chunk if wl.kind == "chunked_prefill" else None)
+        calls = [call]
+        data = "synthetic (seeded host generator)"
+    with ClockSampler(_smi_index(device.index or 0)) as clk:
+        res = time_calls(calls, args, world, device, clk)
+    T = sum(c.T for c in calls)
+    r = rates(wl, calls, res, peaks)
+    roof = r["roofline"]
+    roof["traffic"] = (MLA_TRAFFIC_BYTES_PER_QUERY * T / len(calls)
+                       if (MLA_TRAFFIC_BYTES_PER_QUERY and wl.kind == "prefill" and wl.heads == 128) else None)
     line = {
-        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16+fp8", "data": "synthetic", "config": config,
+        "metric": metric, "value": whole_job_rate(T, world, res["ms_per_step"]), "unit": unit, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16+fp8", "data": data, "config": config,
         "roofline": roof,
-        "stages_ms": {"indexer": idx_ms, "topk": topk_ms, "sparse_mla": mla_ms},
-        "stage_rates": {"indexer_fp8_tflops": idx_tflops, "sparse_mla_bf16_tflops": mla_tflops,
-                        "topk_gbs": (res["idx_pairs"] * 4 + T * wl.k * 4) / (topk_ms / 1e3) / 1e9},
-        "gpu_launches": res["launches_per_step"] * args.steps,
-        "clocks": res["clocks"],
+        "stages_ms": {"indexer": res["stage_ms"][0], "topk": res["stage_ms"][1], "sparse_mla": res["stage_ms"][2]},
+        "stages": r["stages"],
+        "peaks": {"hbm_gbs": peaks["hbm"], "bf16_tflops": peaks["bf16"], "fp8_tflops": peaks["fp8"],
+                  "source": peaks["src"], "fp8_source": peaks["fp8_src"]},
+        "gpu_launches": res["launches"],
+        "clocks": clk.summary(),
     }
-    if res["e2e"]:
-        e = res["e2e"]
+    if ins is not None and not args.no_e2e:
+        e = e2e_headline(calls[0], ins, args, world, device)
         line["e2e"] = {"value": e["value"], "unit": unit, "h2d_bytes_per_step": e["h2d_bytes_per_step"],
                        "d2h_bytes_per_step": e["d2h_bytes_per_step"], "ms_per_step": e["ms_per_step"]}
+    del calls, ins
+    torch.cuda.empty_cache()
+
+    # ---- the other full-size workloads, in the same run
+    if not args.no_extra and not args.seq_len:
+        line["workloads"] = {}
+        for name in ("decode_b64", "decode_128k_mtp2", "chunked_64k"):
+            if name != wl.name:
+                line["workloads"][name] = sub_record(WORKLOADS[name], args, rank, world, device, peaks)
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl)
         line["cpu_baseline"] = {"value": cb["value"], "unit": unit, "cores": cb["cores"], "kind": "oracle",
-                                "sample": f"{cb['rows']} seeded query rows of {wl.name}, full path per row "
-                                          f"(numpy float64), {cb['seconds']:.1f} s"}
+                                "sample": f"{cb['rows']} seeded uniformly random query rows of {wl.name} "
+                                          f"(from a fixed sample of 64), full path per row (numpy float64), "
+                                          f"{cb['seconds']:.1f} s"}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

@@ -18,6 +18,11 @@ sequence for decode.  Cache rows are numbered by position.
 
 Quantisation: N(0,1) float32 values are clamped to +-448 and cast to E4M3 by
 PyTorch's round-to-nearest-even cast; bf16 tensors use PyTorch's RNE cast.
+
+The benchmark's largest workloads (gigabytes of queries and caches) are drawn
+on the device instead (``device_query_tensors``, ``device_cache_tensors``):
+the same distributions and casts from PyTorch's seeded Philox generator.  The
+parity tests use the host streams above.
 """
 from __future__ import annotations
 
@@ -204,3 +209,48 @@ def make_inputs(wl: Workload, seed: int = 0, chunk_index: int | None = None) -> 
         "k_idx": cache_rows(wl, batch, "k_idx", seed),
         "kv": cache_rows(wl, batch, "kv", seed),
     }
+
+
+# ---------------------------------------------------------------------------
+# Device-drawn inputs (benchmark workloads too large to draw on the host)
+# ---------------------------------------------------------------------------
+
+def _device_normal(shape, key: tuple, device, std: float = 1.0):
+    """float32 N(0, std^2) tensor drawn on `device` by PyTorch's Philox generator,
+    seeded from `key` (a tuple of small ints); the same key gives the same values
+    on the same device type."""
+    g = torch.Generator(device=device)
+    h = 0
+    for v in key:
+        h = (h * 1_000_003 + int(v) + 1) % (1 << 63)
+    g.manual_seed(h)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if std != 1.0:
+        x.mul_(std)
+    return x
+
+
+def device_query_tensors(wl: Workload, batch: Batch, device, seed: int = 0, chunk: int = 0) -> dict:
+    """Per-query tensors of one call drawn on the device with the distributions of
+    the host generator (q_I, k_I ~ N(0,1) -> E4M3 after clamping to +-448;
+    w ~ N(0, 1/H_I) fp32; Q ~ N(0,1) -> bf16), keyed by (seed, cfg, tensor, chunk)."""
+    T = batch.num_q
+    qi = _device_normal((T, wl.h_index, D_INDEX), (seed, wl.cfg_id, T_QIDX, chunk), device)
+    w = _device_normal((T, wl.h_index), (seed, wl.cfg_id, T_W, chunk), device, 1.0 / np.sqrt(wl.h_index))
+    q = _device_normal((T, wl.heads, D_QK), (seed, wl.cfg_id, T_Q, chunk), device)
+    return {"q_idx": qi.clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn).view(torch.uint8),
+            "w": w, "q": q.to(torch.bfloat16).view(torch.int16)}
+
+
+def device_cache_tensors(wl: Workload, batch: Batch, device, seed: int = 0) -> dict:
+    """The packed caches of a batch (k_I -> E4M3 bytes [rows, 128], latent rows ->
+    bf16 bits [rows, 576]) drawn on the device, sequence by sequence."""
+    rows = int(batch.kv_len.sum())
+    k_idx = torch.empty((rows, D_INDEX), dtype=torch.uint8, device=device)
+    kv = torch.empty((rows, D_QK), dtype=torch.int16, device=device)
+    for b in range(batch.num_seqs):
+        o, n = int(batch.kv_offset[b]), int(batch.kv_len[b])
+        ki = _device_normal((n, D_INDEX), (seed, wl.cfg_id, T_KIDX, b), device)
+        k_idx[o:o + n] = ki.clamp_(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn).view(torch.uint8)
+        kv[o:o + n] = _device_normal((n, D_QK), (seed, wl.cfg_id, T_KV, b), device).to(torch.bfloat16).view(torch.int16)
+    return {"k_idx": k_idx, "kv": kv}
