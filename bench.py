@@ -501,12 +501,18 @@ def main():
                     help="override the prefill length (smaller cases for profiler captures)")
     ap.add_argument("--chunk", type=int, default=-1,
                     help="chunked workload: time only this chunk's call (default: all chunks)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the number of decode sequences (smaller cases for profiler captures)")
     args = ap.parse_args()
     wl = WORKLOADS[args.config]
     if args.seq_len:
         if wl.kind != "prefill":
             ap.error("--seq-len applies to prefill workloads")
         wl = dataclasses.replace(wl, name=f"{wl.name}@L={args.seq_len}", seq_len=args.seq_len)
+    if args.batch:
+        if wl.kind != "decode":
+            ap.error("--batch applies to decode workloads")
+        wl = dataclasses.replace(wl, name=f"{wl.name}@B={args.batch}", batch=args.batch)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -588,7 +594,7 @@ def main():
     torch.cuda.empty_cache()
 
     # ---- the other full-size workloads, in the same run
-    if not args.no_extra and not args.seq_len:
+    if not args.no_extra and not args.seq_len and not args.batch:
         line["workloads"] = {}
         for name in ("decode_b64", "decode_128k_mtp2", "chunked_64k"):
             if name != wl.name:

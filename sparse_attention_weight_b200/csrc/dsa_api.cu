@@ -93,7 +93,7 @@ int indexer_group(const dsa_batch* b, int H_I) {
 // to fill one wave of the SMs when there are few queries.
 int mla_splits(const dsa_batch* b, int k) {
   const int pairs = num_sms() / 2;
-  const int blocks = (k + 127) / 128;
+  const int blocks = (k + 255) / 256;            // the kernel walks an index row in blocks of 256
   if (b->num_q <= 0) return 1;
   int s = pairs / b->num_q;
   if (s < 1) s = 1;
@@ -179,6 +179,7 @@ dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* 
   p.status = L.status;
   p.G = G;
   p.hi = H_I;
+  p.nacc = G * hp <= 128 ? 4 : 2;
   p.max_kv_len = b->max_kv_len;
   return cuda_status(launch_indexer(tq, tk, p, hp, T, b->num_seqs, b->kv_rows, num_sms(), st));
 }

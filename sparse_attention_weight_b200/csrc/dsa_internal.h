@@ -27,6 +27,7 @@ struct IndexerParams {
   uint32_t* status;
   int G;                     // query tokens per group (N = G * padded H_I)
   int hi;                    // H_I, heads per query token (a multiple of 4, <= 64)
+  int nacc;                  // accumulator buffers in TMEM: 4 when N <= 128, else 2
   int max_kv_len;
 };
 

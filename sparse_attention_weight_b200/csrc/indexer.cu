@@ -26,21 +26,22 @@ namespace dsa {
 
 namespace {
 
-constexpr int kIdxThreads = 320;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;        // four per TMEM lane quadrant, each taking every fourth token
+constexpr int kIdxThreads = 64 + 32 * kEpiWarps;
+constexpr int kMaxAcc = 4;           // accumulator buffers in TMEM (512 columns / N, at most 4)
 constexpr int kKeyTile = 128;        // keys per item (MMA M)
 constexpr int kStages = 6;           // key-tile ring depth
 constexpr int kTileBytes = kKeyTile * DSA_D_INDEX;   // 16 KB
 constexpr int kQBytes = 256 * DSA_D_INDEX;           // 32 KB (N <= 256)
 
 struct __align__(8) IdxSmem {
-  uint8_t q[kQBytes];                  // 1024-aligned (offset 0)
+  uint8_t q[2][kQBytes];               // 1024-aligned (offset 0): query tiles of two groups
   uint8_t k[kStages][kTileBytes];      // 1024-aligned
   float w[kEpiWarps][256];             // per epilogue warp: head weights of the group
-  int32_t n_vis[kEpiWarps][256];       // per epilogue warp: visible keys per token
+  int32_t n_vis[kEpiWarps][64];        // per epilogue warp: visible keys per token (G <= 64)
   uint64_t k_full[kStages], k_empty[kStages];
-  uint64_t q_full, q_empty;
-  uint64_t acc_full[2], acc_empty[2];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t acc_full[kMaxAcc], acc_empty[kMaxAcc];
   uint64_t done;
   uint32_t tmem_base;
   int abort_flag;
@@ -71,14 +72,15 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int i0 = min(total, static_cast<int>(blockIdx.x) * per);
   const int i1 = min(total, i0 + per);
   const int N = p.G * HI;
+  const int nacc = p.nacc;              // accumulator buffers (2 or 4), 512 / nacc columns each
+  const uint32_t acc_cols = 512u / static_cast<uint32_t>(nacc);
   const int hi = p.hi;                  // real heads per token (HI = its padded column stride)
   volatile int* abort_flag = &S.abort_flag;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&S.k_full[s], 1); mbar_init(&S.k_empty[s], 1); }
-    mbar_init(&S.q_full, 1);
-    mbar_init(&S.q_empty, 1);
-    for (int a = 0; a < 2; ++a) { mbar_init(&S.acc_full[a], 1); mbar_init(&S.acc_empty[a], 32 * kEpiWarps); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&S.q_full[b], 1); mbar_init(&S.q_empty[b], 1); }
+    for (int a = 0; a < kMaxAcc; ++a) { mbar_init(&S.acc_full[a], 1); mbar_init(&S.acc_empty[a], 32 * kEpiWarps); }
     mbar_init(&S.done, 1);
     S.abort_flag = 0;
     fence_mbar_init();
@@ -88,7 +90,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (hi != HI) {
     // Tokens are loaded one by one at a stride of HI rows: the HI - hi padding
     // rows of each token stay zero (they meet zero weights in the epilogue).
-    for (int i = threadIdx.x; i < kQBytes / 16; i += blockDim.x)
+    for (int i = threadIdx.x; i < 2 * kQBytes / 16; i += blockDim.x)
       reinterpret_cast<uint4*>(S.q)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
@@ -104,40 +106,41 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (lane == 0) {
         int g = find_group(p.item_off, ngroups, i0);
         int g_lo = p.item_off[g], g_hi = p.item_off[g + 1];
-        int prev_g = -1, issued = 0, q_loads = 0;
+        int prev_g = -1, issued = 0, gq = 0;   // gq: query tiles loaded (buffer gq & 1)
         int64_t row_base = 0;                   // first cache row of the group's sequence
-        uint32_t qe_par = 0;
+        int st = 0;                             // key-ring stage and its phase, advanced per item
+        uint32_t ph = 0;
         for (int i = i0; i < i1; ++i) {
           while (g_hi <= i) { ++g; g_lo = g_hi; g_hi = p.item_off[g + 1]; }
           const int kt = i - g_lo;
           if (g != prev_g) {
             row_base = p.kv_offset[p.group_seq[g]];
-            if (prev_g >= 0) {
-              if (!mbar_wait(&S.q_empty, qe_par, p.status, abort_flag)) break;
-              qe_par ^= 1;
-            }
-            mbar_arrive_expect_tx(&S.q_full, p.G * hi * DSA_D_INDEX);
+            // two query buffers: the tile of group gq reuses the buffer of group
+            // gq - 2, whose MMAs must have completed; the previous group's MMAs may
+            // still be running meanwhile
+            const int qb = gq & 1;
+            if (gq >= 2 && !mbar_wait(&S.q_empty[qb], ((gq - 2) >> 1) & 1, p.status, abort_flag)) break;
+            mbar_arrive_expect_tx(&S.q_full[qb], p.G * hi * DSA_D_INDEX);
             if (hi == HI) {
-              tma_load_2d(S.q, &tm_q, &S.q_full, 0, p.group_q0[g] * HI);
+              tma_load_2d(S.q[qb], &tm_q, &S.q_full[qb], 0, p.group_q0[g] * HI);
             } else {
               for (int u = 0; u < p.G; ++u)     // box = one token's hi rows
-                tma_load_2d(S.q + u * HI * DSA_D_INDEX, &tm_q, &S.q_full, 0, (p.group_q0[g] + u) * hi);
+                tma_load_2d(S.q[qb] + u * HI * DSA_D_INDEX, &tm_q, &S.q_full[qb], 0, (p.group_q0[g] + u) * hi);
             }
-            ++q_loads;
+            ++gq;
             prev_g = g;
           }
-          const int n = i - i0, st = n % kStages;
-          const uint32_t ph = (n / kStages) & 1;
           if (!mbar_wait(&S.k_empty[st], ph ^ 1, p.status, abort_flag)) break;
           mbar_arrive_expect_tx(&S.k_full[st], kTileBytes);
           const int64_t row = row_base + static_cast<int64_t>(kt) * kKeyTile;
           tma_load_2d(S.k[st], &tm_k, &S.k_full[st], 0, static_cast<int>(row));
           ++issued;
+          if (++st == kStages) { st = 0; ph ^= 1; }
         }
         // Never leave with a copy in flight: wait (bounded) for the last load of each stage.
         for (int n = max(0, issued - kStages); n < issued; ++n)
           mbar_wait(&S.k_full[n % kStages], (n / kStages) & 1, p.status, nullptr);
-        if (q_loads > 0) mbar_wait(&S.q_full, (q_loads - 1) & 1, p.status, nullptr);
+        for (int gl = max(0, gq - 2); gl < gq; ++gl) mbar_wait(&S.q_full[gl & 1], (gl >> 1) & 1, p.status, nullptr);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer
@@ -145,34 +148,37 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t idesc = instr_desc(0, 0, false, false, kKeyTile, N);
         int g = find_group(p.item_off, ngroups, i0);
         int g_hi = p.item_off[g + 1];
-        int prev_g = -1;
-        uint32_t qf_par = 0;
+        int prev_g = -1, gm = 0;                // gm: groups started (query buffer (gm - 1) & 1)
+        // Issue must stay lean (this thread shares its scheduler with epilogue
+        // warps): descriptors are built once and stepped by adds to the 14-bit
+        // start-address field (16-byte units); stages advance by counters.
+        const uint64_t kdesc0 = smem_desc_sw128(smem_u32(S.k[0]), 16, 1024);
+        const uint64_t qdesc0 = smem_desc_sw128(smem_u32(S.q[0]), 16, 1024);
+        uint64_t qd = qdesc0, kd = kdesc0;
+        uint32_t d = tmem;
+        int st = 0, a = 0;
+        uint32_t ph = 0, aph = 0;
         for (int i = i0; i < i1; ++i) {
           while (g_hi <= i) { ++g; g_hi = p.item_off[g + 1]; }
           if (g != prev_g) {
-            if (!mbar_wait(&S.q_full, qf_par, p.status, abort_flag)) break;
-            qf_par ^= 1;
+            if (!mbar_wait(&S.q_full[gm & 1], (gm >> 1) & 1, p.status, abort_flag)) break;
+            qd = qdesc0 + static_cast<uint64_t>((gm & 1) * (kQBytes / 16));
+            ++gm;
             prev_g = g;
           }
-          const int n = i - i0, st = n % kStages, a = n & 1;
-          const uint32_t ph = (n / kStages) & 1, aph = (n >> 1) & 1;
           if (!mbar_wait(&S.acc_empty[a], aph ^ 1, p.status, abort_flag)) break;
           tc_fence_after();
           if (!mbar_wait(&S.k_full[st], ph, p.status, abort_flag)) break;
           tc_fence_after();
-          const uint32_t a_base = smem_u32(S.k[st]);
-          const uint32_t b_base = smem_u32(S.q);
-          const uint32_t d = tmem + a * 256;
 #pragma unroll
-          for (int kk = 0; kk < DSA_D_INDEX / 32; ++kk) {
-            const uint64_t ad = smem_desc_sw128(a_base + kk * 32, 16, 1024);
-            const uint64_t bd = smem_desc_sw128(b_base + kk * 32, 16, 1024);
-            umma_f8(d, ad, bd, idesc, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < DSA_D_INDEX / 32; ++kk)
+            umma_f8(d, kd + static_cast<uint64_t>(kk * 2), qd + static_cast<uint64_t>(kk * 2), idesc, kk > 0 ? 1u : 0u);
           umma_commit(&S.k_empty[st]);
           umma_commit(&S.acc_full[a]);
           const bool last_of_group = (i + 1 == i1) || (g_hi <= i + 1);
-          if (last_of_group) umma_commit(&S.q_empty);
+          if (last_of_group) umma_commit(&S.q_empty[(gm - 1) & 1]);
+          if (++st == kStages) { st = 0; ph ^= 1; kd = kdesc0; } else { kd += kTileBytes / 16; }
+          if (++a == nacc) { a = 0; aph ^= 1; d = tmem; } else { d += acc_cols; }
         }
         umma_commit(&S.done);
         mbar_wait(&S.done, 0, p.status, nullptr);
@@ -180,15 +186,17 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     } else {
       // ------------------------------------------------------------ epilogue
       // Warp-uniform control flow: lane 0 waits on barriers, the warp follows.
-      const int ew = warp - 2;                    // 0..7
+      const int ew = warp - 2;                    // 0..15
       const int quad = warp & 3;                  // TMEM lane quadrant of this warp
-      const int tsub = ew >> 2;                   // token parity handled by this warp
+      const int tsub = ew >> 2;                   // tokens tsub, tsub + 4, ... of each group
       const int row = quad * 32 + lane;           // key within the tile
       float* sw = S.w[ew];
       int32_t* snv = S.n_vis[ew];
       int g = find_group(p.item_off, ngroups, i0);
       int g_lo = p.item_off[g], g_hi = p.item_off[g + 1];
       int prev_g = -1, cnt = 0, q0 = 0;
+      int a = 0;                                  // accumulator buffer and its phase, advanced per item
+      uint32_t aph = 0;
       for (int i = i0; i < i1; ++i) {
         while (g_hi <= i) { ++g; g_lo = g_hi; g_hi = p.item_off[g + 1]; }
         const int kt = i - g_lo;
@@ -196,46 +204,73 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           __syncwarp();
           q0 = p.group_q0[g];
           cnt = p.group_cnt[g];
-          for (int j = lane; j < cnt * HI; j += 32) {
-            const int tok = j / HI, h = j - tok * HI;
-            sw[j] = h < hi ? p.w[static_cast<int64_t>(q0 + tok) * hi + h] : 0.f;
+          // all loads of the group's weights and visible counts in flight at once
+          constexpr int kWPer = 256 / 32;         // G * HI <= 256
+          float wv[kWPer];
+          int nv[2];
+#pragma unroll
+          for (int u = 0; u < kWPer; ++u) {
+            const int j = lane + 32 * u, tok = j / HI, h = j - tok * HI;
+            wv[u] = (j < cnt * HI && h < hi) ? __ldg(p.w + static_cast<int64_t>(q0 + tok) * hi + h) : 0.f;
           }
-          for (int j = lane; j < cnt; j += 32) snv[j] = max(0, p.q_nvis[q0 + j]);
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int j = lane + 32 * u;
+            nv[u] = j < cnt ? __ldg(p.q_nvis + q0 + j) : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < kWPer; ++u) sw[lane + 32 * u] = wv[u];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) snv[lane + 32 * u] = max(0, nv[u]);   // cnt <= 64
           __syncwarp();
           prev_g = g;
         }
-        const int n = i - i0, a = n & 1;
-        const uint32_t aph = (n >> 1) & 1;
         int ok = 1;
         if (lane == 0) ok = mbar_wait(&S.acc_full[a], aph, p.status, abort_flag) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
         const int s = kt * kKeyTile + row;
-        const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + a * 256;
+        const uint32_t tbase = tmem + (static_cast<uint32_t>(quad * 32) << 16) + a * acc_cols;
         if constexpr (HI >= 32) {
-          for (int tok = tsub; tok < cnt; tok += 2) {
-            uint32_t v[HI];
-#pragma unroll
-            for (int c = 0; c < HI / 32; ++c)
-              tmem_ld32(tbase + tok * HI + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
-            tmem_ld_wait();
+          // one token per pass: its HI head columns, ReLU, then the weighted head
+          // sum in packed pairs (fma.rn.f32x2) over four independent accumulators
+          for (int tok = tsub; tok < cnt; tok += 4) {
             const float* wr = &sw[tok * HI];
-            float acc0 = 0.f, acc1 = 0.f;
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int j = 0; j < HI; j += 4) {
-              const float4 w4 = *reinterpret_cast<const float4*>(wr + j);
-              acc0 = fmaf(w4.x, fmaxf(__uint_as_float(v[j + 0]), 0.f), acc0);
-              acc1 = fmaf(w4.y, fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
-              acc0 = fmaf(w4.z, fmaxf(__uint_as_float(v[j + 2]), 0.f), acc0);
-              acc1 = fmaf(w4.w, fmaxf(__uint_as_float(v[j + 3]), 0.f), acc1);
+            for (int c = 0; c < HI / 32; ++c) {      // 32 head columns per TMEM load
+              uint32_t v[32];
+              tmem_ld32(tbase + tok * HI + c * 32, v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                const float4 wa = *reinterpret_cast<const float4*>(wr + c * 32 + j);
+                const float4 wb = *reinterpret_cast<const float4*>(wr + c * 32 + j + 4);
+                const int u = (j >> 3) & 1;
+                acc[2 * u] = ffma2(make_float2(wa.x, wa.y),
+                                   make_float2(fmaxf(__uint_as_float(v[j + 0]), 0.f), fmaxf(__uint_as_float(v[j + 1]), 0.f)),
+                                   acc[2 * u]);
+                acc[2 * u + 1] = ffma2(make_float2(wa.z, wa.w),
+                                       make_float2(fmaxf(__uint_as_float(v[j + 2]), 0.f), fmaxf(__uint_as_float(v[j + 3]), 0.f)),
+                                       acc[2 * u + 1]);
+                acc[2 * u] = ffma2(make_float2(wb.x, wb.y),
+                                   make_float2(fmaxf(__uint_as_float(v[j + 4]), 0.f), fmaxf(__uint_as_float(v[j + 5]), 0.f)),
+                                   acc[2 * u]);
+                acc[2 * u + 1] = ffma2(make_float2(wb.z, wb.w),
+                                       make_float2(fmaxf(__uint_as_float(v[j + 6]), 0.f), fmaxf(__uint_as_float(v[j + 7]), 0.f)),
+                                       acc[2 * u + 1]);
+              }
             }
-            if (s < snv[tok]) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = acc0 + acc1;
+            const float sum = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                              ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+            if (s < snv[tok]) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = sum;
           }
         } else {
           constexpr int TPC = 32 / HI;             // tokens per 32-column chunk
           const int nchunks = (cnt * HI + 31) / 32;
-          for (int c = tsub; c < nchunks; c += 2) {
+          for (int c = tsub; c < nchunks; c += 4) {
             uint32_t v[32];
             tmem_ld32(tbase + c * 32, v);
             tmem_ld_wait();
@@ -256,6 +291,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         tc_fence_before();
         mbar_arrive(&S.acc_empty[a]);
+        if (++a == nacc) { a = 0; aph ^= 1; }
       }
     }
   }

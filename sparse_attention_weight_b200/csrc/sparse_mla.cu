@@ -9,37 +9,42 @@
 // Per query token the state is large: Q is 128 heads x 576 (144 KB bf16) and
 // the output accumulator 128 x 512 fp32 (256 KB, all of one SM's TMEM).  So a
 // token is handled by a CTA pair (a 2-CTA cluster) using the pair form of the
-// tensor-core MMA (cta_group::2, M = 128 = 64 heads per CTA):
-//   S  = Q K^T : A = the CTA's 64 heads of Q (72 KB, resident), B = a block of
-//                128 gathered rows, split 64/64 between the CTAs (K-major);
-//                per CTA: 64 heads x 128 rows fp32 in TMEM (64 columns).
-//   O += P V   : A = P (64 heads x 128 rows, bf16, written by the softmax
-//                warps), B = V rows of the block, each CTA holding 128 of every
-//                256 value dims (MN-major); per CTA: 64 heads x 512 dims fp32
-//                (256 TMEM columns).
+// tensor-core MMA (cta_group::2, M = 128 = 64 heads per CTA), over blocks of
+// 256 selected rows, 128 gathered by each CTA:
+//   S  = Q K^T : A = the CTA's 64 heads of Q (72 KB, resident), B = the block's
+//                256 rows (K-major), N = 256; per CTA: 64 heads x 256 rows fp32
+//                in TMEM (128 columns).
+//   O += P V   : A = P (64 heads x 256 rows, bf16, K-major, written by the
+//                softmax warps), B = V rows of the block, each CTA holding 128
+//                of every 256 value dims (MN-major), N = 256; per CTA: 64 heads
+//                x 512 dims fp32 (256 TMEM columns).
+// A single tcgen05.mma takes longer to issue (about 58 ns) than a pair MMA of
+// 64 x 128 per SM takes to execute, so the block is 256 rows wide: every S
+// and PV instruction then moves 64 x 256 per SM, and a block needs 68 of them.
 // S is double buffered in TMEM, so the tensor core computes S of block j+1
 // while the softmax warps turn S of block j into P.  The softmax keeps a
 // reference maximum per head and rescales O (in TMEM) only when a block's
 // maximum exceeds it by more than 2^8, so P stays <= 256 and most blocks skip
-// the rescale.  Rows are gathered from L2 by index with 16-byte cp.async (8
-// lanes per 128-byte row segment: coalesced) into 128-byte-swizzled tiles, once:
-// each CTA gathers its 64 rows x 576 dims for S, and the V operand (the first
-// 512 of those dims, needed by both CTAs, each for its value dims) is copied
-// out of the S rings by bulk shared-memory copies across the pair.  Gathering
-// V from L2 a second time nearly doubled the gather traffic, and the gathers'
-// latency, not the tensor core, set the pace.
+// the rescale.
 //
-// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-11 gather of the
-// S operand rows, 12 TMEM owner and (in the even CTA) issuer of the S MMAs,
-// 13 Q load and S relay, 14 V copier and relay, 15 (even CTA) issuer of the
+// Rows are gathered from L2 by index with 16-byte cp.async (8 lanes per 128-byte
+// row segment: coalesced) into 128-byte-swizzled tiles.  Two streaming rings
+// decouple the gathers from the MMAs: the S ring holds 64-dim chunks of the
+// CTA's 128 rows (16 KB slots, refilled as soon as the S MMAs read them) and
+// the V ring holds 32-row slices of the block with the CTA's value dims (16 KB
+// slots, refilled as soon as the PV MMAs read them).  Each CTA thus reads the
+// value dims it multiplies straight from L2; no V data crosses the pair.
+//
+// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-7 gathers of the S
+// ring, 8-11 gathers of the V ring, 12 TMEM owner and (in the even CTA) issuer
+// of the S MMAs, 13 Q load and S relay, 14 V relay, 15 (even CTA) issuer of the
 // PV MMAs.  Signals from the odd CTA to the even CTA's barriers are
 // asynchronous 4-byte stores counted as transaction bytes (a thread-level
-// remote mbarrier arrive stalls its thread for a round trip, which throttled
-// the gathers when every stage used one).  Gather threads never wait for their
-// own copies: each arrives on a local stage barrier through
-// cp.async.mbarrier.arrive (hardware-tracked completion), and a relay lane
-// that has no copies in flight forwards the completed stage to the even CTA's
-// barrier, which the MMA issuer waits on.
+// remote mbarrier arrive stalls its thread for a round trip).  Gather threads
+// never wait for their own copies: each arrives on a local stage barrier
+// through cp.async.mbarrier.arrive (hardware-tracked completion), and a relay
+// lane that has no copies in flight forwards the completed stage to the even
+// CTA's barrier, which the MMA issuer waits on.
 #include <cuda_bf16.h>
 
 #include "dsa_common.cuh"
@@ -50,35 +55,37 @@ namespace dsa {
 namespace {
 
 constexpr int kMlaThreads = 512;
-constexpr int kGatherWarps = 8;         // S-ring gather warps; each loads 8 rows of every chunk
-constexpr int kBlk = 128;             // selected rows per block (pair)
-constexpr int kHalf = 64;             // rows per CTA for the S operand; heads per CTA
+constexpr int kSWarps = 4;            // S-ring gather warps: 32 rows of every chunk each
+constexpr int kVWarps = 4;            // V-ring gather warps: 8 rows of every slice each
+constexpr int kBlk = 256;             // selected rows per block (pair)
+constexpr int kRows = 128;            // rows per CTA per block (S operand)
+constexpr int kHeads = 64;            // heads per CTA
 constexpr int kDChunks = DSA_D_QK / 64;   // 9 chunks of 64 dims
-constexpr int kSStages = 9;           // S-operand ring (8 KB slots): one full block
-constexpr int kVChunks = 8;           // value dims 0..511 = S-ring chunks 0..7
+constexpr int kSStages = 4;           // S ring: 16 KB slots (128 rows x 64 dims)
+constexpr int kVRows = 32;            // rows per V slice
+constexpr int kVSlices = kBlk / kVRows;   // 8 slices per block
+constexpr int kVStages = 3;           // V ring: 16 KB slots (32 rows x 256 value dims)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-constexpr uint32_t kSCol = 0;         // TMEM columns [0,128): two S buffers of 64
-constexpr uint32_t kOCol = 128;       // TMEM columns [128,384): O (2 x 128)
+constexpr uint32_t kSCol = 0;         // TMEM columns [0,256): two S buffers of 128
+constexpr uint32_t kOCol = 256;       // TMEM columns [256,512): O (2 x 128)
 
 struct MlaSmem {
-  uint8_t q[kDChunks][kHalf * 128];          // 72 KB  Q of this CTA's heads (K-major SW128)
-  uint8_t s_ring[kSStages][kHalf * 128];     // 72 KB  S operand chunks: 64 rows x 64 dims
-  uint8_t vbuf[4][kBlk * 128];               // 64 KB  V operand: 4 dim groups x 128 rows (MN-major SW128)
-  uint8_t p[2][kHalf * 128];                 // 16 KB  P: 64 heads x 128 rows (two K chunks)
+  uint8_t q[kDChunks][kHeads * 128];         // 72 KB  Q of this CTA's heads (K-major SW128)
+  uint8_t s_ring[kSStages][kRows * 128];     // 64 KB  S operand chunks: 128 rows x 64 dims
+  uint8_t v_ring[kVStages][4][kVRows * 128]; // 48 KB  V slices: 4 dim groups x 32 rows (MN-major SW128)
+  uint8_t p[kBlk / 64][kHeads * 128];        // 32 KB  P: 64 heads x 256 rows (four K chunks of 64 rows)
   float xmax[2][128];
   float lsum[128];
   uint32_t valid[2048 / 32];                 // bit e: entry e of the index row is a usable row
   uint64_t q_full, q_ready;
   uint64_t s_full[kSStages], s_empty[kSStages], s_loaded[kSStages];
-  uint64_t v_full[2], v_empty[2];            // per quarter q: V-buffer dim groups 2q, 2q+1 (all rows)
-  uint64_t v_loaded[2][2];                   // tiles of half h, dim groups 2q and 2q+1, landed here
-  uint64_t xfer[2];                          // this CTA's copies of value chunks 4q..4q+3 landed in both CTAs
+  uint64_t v_full[kVStages], v_empty[kVStages], v_loaded[kVStages];
   uint64_t s_ready[2], s_free[2];
   uint64_t p_full, p_empty;
   uint64_t mx_bar[2], l_bar;
   uint64_t done;
   // mailboxes of the peer CTA's asynchronous signals (contents unused)
-  uint32_t mbox_q, mbox_s[kSStages], mbox_v[2], mbox_x[2], mbox_sfree[2][4], mbox_pfull[4];
+  uint32_t mbox_q, mbox_s[kSStages], mbox_v[kVStages], mbox_sfree[2][4], mbox_pfull[4];
   uint32_t tmem_base;
   int last_used[8];                          // per prologue warp: last usable entry, -1 if none
   int abort_flag;
@@ -103,22 +110,6 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // Arrive on `bar` once every cp.async issued so far by this thread has completed.
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Address of the same shared-memory object in CTA `cta` of the cluster.
-__device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t cta) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(cta));
-  return r;
-}
-
-// Bulk copy of `bytes` from this CTA's shared memory to `dst`, a shared::cluster
-// address in this CTA or its peer; the bytes are counted on `bar`, a barrier in
-// the destination CTA.
-__device__ __forceinline__ void bulk_copy_s2c(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
-               : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
@@ -149,9 +140,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
 }
 
 // Order in which the chunks of a block are gathered, forwarded and multiplied:
-// the RoPE chunk (dims 512..575) first, since its slot is free as soon as the
-// previous block's S MMA read it, then the value chunks 0..7, whose slots also
-// wait for their copies into the V buffers.
+// the RoPE chunk (dims 512..575) first, then the value chunks 0..7.
 __device__ __forceinline__ int chunk_at(int i) { return i == 0 ? kDChunks - 1 : i - 1; }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMlaThreads, 1)
@@ -177,12 +166,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
     mbar_init(&S.q_full, 1);
     mbar_init(&S.q_ready, 1);
     for (int i = 0; i < kSStages; ++i) {
-      mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], kGatherWarps * 32);
+      mbar_init(&S.s_full[i], 1); mbar_init(&S.s_empty[i], 1); mbar_init(&S.s_loaded[i], kSWarps * 32);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1);
-      mbar_init(&S.v_loaded[i][0], 1); mbar_init(&S.v_loaded[i][1], 1);
-      mbar_init(&S.xfer[i], 1);                 // own arrival (+4 tx bytes from the peer's report)
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], kVWarps * 32);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 4); mbar_init(&S.mx_bar[i], 128);
@@ -228,7 +215,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
-  // blocks of 128 entries covering the used part of the index row, split evenly
+  // blocks of 256 entries covering the used part of the index row, split evenly
   int nblk = 0, blk0 = 0;
   {
     int last = -1;
@@ -241,43 +228,38 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
   }
 
   const int H = p.H;
-  const int head0 = static_cast<int>(rank) * kHalf;        // first head of this CTA
+  const int head0 = static_cast<int>(rank) * kHeads;       // first head of this CTA
 
   if (nblk > 0) {
     if (warp < 4) {
       // ================================================================ softmax
-      const int tid = threadIdx.x;                           // TMEM lane
-      const int hl = tid & 63;                               // local head
-      const int half = tid >> 6;                             // which 64 rows of each block
+      // Thread = TMEM lane: head hl of this CTA, over the 128 rows gathered by
+      // CTA `half` (the S tile's columns 128*half .. +127 sit on lanes 64*half ..).
+      const int tid = threadIdx.x;
+      const int hl = tid & 63;
+      const int half = tid >> 6;
       const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < nblk; ++j) {
         const int sb = j & 1;
         const uint32_t sph = (j >> 1) & 1;
-        // validity of this warp's 64 columns
-        const int pos0 = (blk0 + j) * kBlk + half * 64;      // multiple of 64
-        const uint32_t vm0 = pos0 < 2048 ? S.valid[pos0 >> 5] : 0u;
-        const uint32_t vm1 = pos0 + 32 < 2048 ? S.valid[(pos0 >> 5) + 1] : 0u;
+        // validity of this thread's 128 entries (four 32-bit words)
+        const int pos0 = (blk0 + j) * kBlk + half * kRows;   // multiple of 128
+        auto valid_word = [&](int c) -> uint32_t { return pos0 + 32 * c < 2048 ? S.valid[(pos0 >> 5) + c] : 0u; };
         if (!warp_wait(&S.s_ready[sb], sph, p.status, ab, false)) break;
         tc_fence_after();
-        uint32_t sr[64];
-        {
-          uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-          uint32_t (&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-          tmem_ld32(tmem + lane_addr + kSCol + sb * 64, a);
-          tmem_ld32(tmem + lane_addr + kSCol + sb * 64 + 32, b);
-          tmem_ld_wait();
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) pair_signal(rank, &S.s_free[sb], &S.mbox_sfree[sb][warp], warp == 0, 16);
-        float* x = reinterpret_cast<float*>(sr);             // logits in log2 units, in place
+        const uint32_t sbase = tmem + lane_addr + kSCol + sb * 128;
+        // pass 1: this thread's maximum over its 128 logits (log2 units)
         float mloc = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(sbase + c * 32, sr);
+          const uint32_t vmc = valid_word(c);
+          tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const bool v = ((c < 32 ? vm0 >> c : vm1 >> (c - 32)) & 1u) != 0;
-          x[c] = v ? __uint_as_float(sr[c]) * p.sm_scale_log2 : -INFINITY;
-          mloc = fmaxf(mloc, x[c]);
+          for (int u = 0; u < 32; ++u)
+            if ((vmc >> u) & 1u) mloc = fmaxf(mloc, __uint_as_float(sr[u]) * p.sm_scale_log2);
         }
         // pair maximum of this head over the whole block
         S.xmax[sb][tid] = mloc;
@@ -289,20 +271,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         // a head with no usable entry so far has m_new = -inf and every x = -inf:
         // subtract 0 instead, so that each p is 2^-inf = 0 (never -inf - -inf)
         const float msub = m_new == -INFINITY ? 0.f : m_new;
-        // The denominator sums the bf16-rounded weights that the PV MMA multiplies
-        // V by, so the output is a convex combination of the selected rows.
-        float psum = 0.f;
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = ex2_approx(x[c] - msub);
-          const float p1 = ex2_approx(x[c + 1] - msub);
-          const uint32_t pp = pack_bf16(p0, p1);
-          psum += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
-          pk[c >> 1] = pp;
-        }
         const float alpha = rescale ? ex2_approx(m_ref - m_new) : 1.f;   // m_ref = -inf -> 0
-        l = l * alpha + psum;
         // P buffer and O are free once PV of the previous block completed
         if (j > 0) {
           if (!warp_wait(&S.p_empty, (j - 1) & 1, p.status, ab, false)) break;
@@ -322,18 +291,39 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
           }
         }
         m_ref = m_new;
-        // P row hl, K chunk `half` (rows half*64 .. +63 of the block), 128B-swizzled
-        {
-          uint8_t* prow = S.p[half] + hl * 128;
+        // pass 2: P = 2^(x - m) in bf16, written as P row hl of K chunks 2*half and
+        // 2*half+1 (rows 128*half .. +127 of the block), 128B-swizzled; the
+        // denominator sums the same bf16 values that the PV MMA multiplies V by
+        float psum = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(sbase + c * 32, sr);
+          const uint32_t vmc = valid_word(c);
+          tmem_ld_wait();
+          uint32_t pk[16];
 #pragma unroll
-          for (int c16 = 0; c16 < 8; ++c16) {
-            const uint32_t off = static_cast<uint32_t>(((c16 ^ (hl & 7)) << 4));
-            *reinterpret_cast<uint4*>(prow + off) =
-                make_uint4(pk[c16 * 4 + 0], pk[c16 * 4 + 1], pk[c16 * 4 + 2], pk[c16 * 4 + 3]);
+          for (int u = 0; u < 32; u += 2) {
+            const float x0 = ((vmc >> u) & 1u) ? __uint_as_float(sr[u]) * p.sm_scale_log2 : -INFINITY;
+            const float x1 = ((vmc >> (u + 1)) & 1u) ? __uint_as_float(sr[u + 1]) * p.sm_scale_log2 : -INFINITY;
+            const uint32_t pp = pack_bf16(ex2_approx(x0 - msub), ex2_approx(x1 - msub));
+            psum += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
+            pk[u >> 1] = pp;
+          }
+          uint8_t* prow = S.p[half * 2 + (c >> 1)] + hl * 128;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int c16 = (c & 1) * 4 + q4;                // 16-byte chunk of the 128-byte row
+            *reinterpret_cast<uint4*>(prow + ((c16 ^ (hl & 7)) << 4)) =
+                make_uint4(pk[q4 * 4 + 0], pk[q4 * 4 + 1], pk[q4 * 4 + 2], pk[q4 * 4 + 3]);
           }
         }
-        fence_proxy_async_smem();
+        l = l * alpha + psum;
+        // S buffer sb has been read: the S MMAs of block j+2 may overwrite it
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) pair_signal(rank, &S.s_free[sb], &S.mbox_sfree[sb][warp], warp == 0, 16);
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) pair_signal(rank, &S.p_full, &S.mbox_pfull[warp], warp == 0, 16);
       }
@@ -391,54 +381,86 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
             p.part_lse[(static_cast<int64_t>(t) * p.splits + split) * H + h] = lse_v;
         }
       }
-    } else if (warp < 12) {
-      // ================================================================ gathers
-      // Warps 4-11 fill the S ring together, chunk by chunk in chunk_at order:
-      // warp w loads rows 8w..8w+7 of this CTA's 64 (two 16-byte copies per lane
+    } else if (warp < 4 + kSWarps) {
+      // ================================================================ S gathers
+      // Warps 4-7 fill the S ring, chunk by chunk in chunk_at order: warp w
+      // loads rows 32w..32w+31 of this CTA's 128 (eight 16-byte copies per lane
       // per chunk, 8 lanes per 128-byte row segment) and every lane signals with
-      // one hardware-tracked arrive.  Issuing a chunk across all eight warps
-      // makes chunks land one after another, so the S MMAs and the V copies start
-      // on the first chunk while the rest are in flight (chunk-per-warp issue
-      // made a block's chunks land together, at the end of its burst).  A value
-      // chunk's slot is refilled once its copies of the previous block landed.
+      // one hardware-tracked arrive.  A slot is refilled as soon as the S MMAs
+      // have read it.
       const int gw = warp - 4;
       const int c16 = lane & 7;
       const int rsub = lane >> 3;
-      // local row indices of this lane's two rows (8gw + rsub, 8gw + 4 + rsub) of block b
-      auto rows_of = [&](int b, int (&rr)[2]) {
+      // local row indices of this lane's rows (32gw + 4i + rsub) of block b
+      auto rows_of = [&](int b, int (&rr)[8]) {
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int e = b * kBlk + static_cast<int>(rank) * kHalf + 8 * gw + 4 * i + rsub;
+        for (int i = 0; i < 8; ++i) {
+          const int e = b * kBlk + static_cast<int>(rank) * kRows + 32 * gw + 4 * i + rsub;
           const int v = e < p.k ? __ldg(idx_row + e) : -1;
           rr[i] = (v >= 0 && v < len) ? v : -1;
         }
       };
-      int cur[2], nxt[2] = {-1, -1};
+      int cur[8], nxt[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) nxt[i] = -1;
       rows_of(blk0, cur);
+      int slot = 0;
+      uint32_t sph = 0;
       for (int j = 0; j < nblk; ++j) {
         if (j + 1 < nblk) rows_of(blk0 + j + 1, nxt);
         bool ok = true;
         for (int i = 0; i < kDChunks; ++i) {
           const int c = chunk_at(i);
-          if (!warp_wait(&S.s_empty[c], (j & 1) ^ 1, p.status, ab, false)) { ok = false; break; }
-          // value chunks 4q..4q+3 (i = 4q+1..): their copies of block j-1 must have landed
-          if ((i == 1 || i == 5) && j > 0 && !warp_wait(&S.xfer[i >> 2], (j - 1) & 1, p.status, ab, false)) {
-            ok = false;
-            break;
-          }
-          const uint32_t dst0 = smem_u32(S.s_ring[c]);
+          if (!warp_wait(&S.s_empty[slot], sph ^ 1, p.status, ab, false)) { ok = false; break; }
+          const uint32_t dst0 = smem_u32(S.s_ring[slot]);
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int r = 8 * gw + 4 * h + rsub;               // row within this CTA's 64
+          for (int h = 0; h < 8; ++h) {
+            const int r = 32 * gw + 4 * h + rsub;              // row within this CTA's 128
             const int v = cur[h];
             cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4),
                        p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + c * 64 + c16 * 8, v < 0 ? 0u : 16u);
           }
-          cp_async_arrive_noinc(&S.s_loaded[c]);
+          cp_async_arrive_noinc(&S.s_loaded[slot]);
+          if (++slot == kSStages) { slot = 0; sph ^= 1; }
         }
         if (!ok) break;
-        cur[0] = nxt[0];
-        cur[1] = nxt[1];
+#pragma unroll
+        for (int h = 0; h < 8; ++h) cur[h] = nxt[h];
+      }
+      cp_async_wait_all();
+    } else if (warp < 4 + kSWarps + kVWarps) {
+      // ================================================================ V gathers
+      // Warps 8-11 gather the V operand straight from L2, slice by slice: a slice
+      // is 32 rows of the block (both CTAs' rows) with this CTA's value dims,
+      // dim group g (0..3) = dims (g/2)*256 + r*128 + (g%2)*64 (MN-major SW128:
+      // one 128-byte line per row and group).  Warp w loads rows 8w..8w+7 of
+      // the slice, one 16-byte copy per lane and row (lane = group * 8 + chunk).
+      // A slot is refilled as soon as the PV MMAs have read it.
+      const int vw = warp - 4 - kSWarps;
+      const int g = lane >> 3;
+      const int c16 = lane & 7;
+      const int dim0 = (g >> 1) * 256 + static_cast<int>(rank) * 128 + (g & 1) * 64 + c16 * 8;
+      int slot = 0;
+      uint32_t vph = 0;
+      bool ok = true;
+      for (int j = 0; j < nblk && ok; ++j) {
+        for (int vs = 0; vs < kVSlices; ++vs) {
+          // indices of rows 8vw .. 8vw+7 of the slice: lane r < 8 loads row r, then broadcast
+          const int e = (blk0 + j) * kBlk + vs * kVRows + 8 * vw + (lane & 7);
+          int mine = e < p.k ? __ldg(idx_row + e) : -1;
+          mine = (mine >= 0 && mine < len) ? mine : -1;
+          if (!warp_wait(&S.v_empty[slot], vph ^ 1, p.status, ab, false)) { ok = false; break; }
+          const uint32_t dst0 = smem_u32(S.v_ring[slot][g]);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int v = __shfl_sync(0xffffffffu, mine, i);
+            const int r = 8 * vw + i;                          // row of the slice
+            cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4),
+                       p.kv + (v < 0 ? 0 : base + v) * DSA_D_QK + dim0, v < 0 ? 0u : 16u);
+          }
+          cp_async_arrive_noinc(&S.v_loaded[slot]);
+          if (++slot == kVStages) { slot = 0; vph ^= 1; }
+        }
       }
       cp_async_wait_all();
     } else if (warp == 13 && lane == 0) {
@@ -446,132 +468,95 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       // This CTA's Q load (9 TMA boxes of 64 dims x 64 heads), then completed
       // S-ring stages forwarded, in order, to the even CTA's barriers.  It waits
       // with the suspending try_wait: a spinning test_wait poller competes with
-      // the gathers for the shared-memory pipe.  As in cp.async-fed tensor-core
-      // pipelines, the stage barrier (completed by the copies themselves) orders
-      // the data before the MMA that reads it.
-      mbar_arrive_expect_tx(&S.q_full, kDChunks * kHalf * 128);
+      // the gathers for the shared-memory pipe.
+      mbar_arrive_expect_tx(&S.q_full, kDChunks * kHeads * 128);
       for (int dc = 0; dc < kDChunks; ++dc)
         tma_load_2d(S.q[dc], &tm_q, &S.q_full, dc * 64, t * H + head0);
       if (mbar_wait(&S.q_full, 0, p.status, ab)) pair_signal(rank, &S.q_ready, &S.mbox_q, true, 4);
-      for (int i = 0; i < nblk * kDChunks; ++i) {
-        const int c = chunk_at(i % kDChunks);
-        if (!mbar_wait(&S.s_loaded[c], (i / kDChunks) & 1, p.status, ab)) break;
-        pair_signal(rank, &S.s_full[c], &S.mbox_s[c], true, 4);
+      int slot = 0;
+      uint32_t sph = 0;
+      for (int gi = 0; gi < nblk * kDChunks; ++gi) {
+        if (!mbar_wait(&S.s_loaded[slot], sph, p.status, ab)) break;
+        fence_proxy_async_smem();                            // cp.async writes -> tensor-core reads
+        pair_signal(rank, &S.s_full[slot], &S.mbox_s[slot], true, 4);
+        if (++slot == kSStages) { slot = 0; sph ^= 1; }
       }
     } else if (warp == 14 && lane == 0) {
-      // ================================================================ V copier / relay
-      // The V operand is the first 512 dims of the rows already in the S rings,
-      // so it is never gathered from L2 twice: this CTA's rows (half `rank` of
-      // the block) are copied, chunk by chunk, from its S ring into the V
-      // buffers, its own dims groups into its own buffer and the peer's into the
-      // peer's (bulk shared-memory copies over the cluster).  V buffer dim group
-      // g of CTA r holds dims (g/2)*256 + r*128 + (g%2)*64, i.e. S chunk
-      // 4*(g/2) + 2r + g%2; every row is a 128-byte swizzled line in both layouts,
-      // so a tile copies verbatim.  Value chunks go in two quarters (chunks
-      // 4q..4q+3 = dim groups 2q, 2q+1 of both CTAs): once a quarter's tiles have
-      // landed here the lane reports it to the even CTA (v_full, for the PV MMAs)
-      // and to the CTAs whose rows they are (xfer: those S slots may be refilled),
-      // while the next quarter is still being copied.
-      const uint32_t peer = rank ^ 1u;
-      for (int j = 0; j < nblk; ++j) {
-        bool ok = true;
-        for (int h = 0; h < 2; ++h)
-          for (int q = 0; q < 2; ++q) mbar_arrive_expect_tx(&S.v_loaded[h][q], 2 * kHalf * 128);
-        for (int q = 0; q < kVChunks / 4 && ok; ++q) {
-          // quarter q of the V buffers is free once the PV MMAs of block j-1 on it completed
-          if (j > 0 && !mbar_wait(&S.v_empty[q], (j - 1) & 1, p.status, ab)) { ok = false; break; }
-          for (int c = 4 * q; c < 4 * q + 4; ++c) {
-            if (!mbar_wait(&S.s_loaded[c], j & 1, p.status, ab)) { ok = false; break; }
-            fence_proxy_async_smem();                        // cp.async writes -> bulk-copy reads
-            const uint32_t owner = static_cast<uint32_t>((c >> 1) & 1);   // CTA whose dims these are
-            const int g = (c >> 2) * 2 + (c & 1);
-            const uint32_t dst = smem_u32(&S.vbuf[g][static_cast<int>(rank) * kHalf * 128]);
-            const uint32_t bar = smem_u32(&S.v_loaded[rank][q]);
-            if (owner == rank) bulk_copy_s2c(dst, smem_u32(S.s_ring[c]), kHalf * 128, bar);
-            else bulk_copy_s2c(mapa(dst, peer), smem_u32(S.s_ring[c]), kHalf * 128, mapa(bar, peer));
-          }
-          for (int h = 0; h < 2 && ok; ++h) {
-            if (!mbar_wait(&S.v_loaded[h][q], j & 1, p.status, ab)) { ok = false; break; }
-            // tiles of half h hold CTA h's rows: tell CTA h these copies of its chunks landed
-            // (own copies: this CTA's arrival, which also expects the peer's report;
-            // the peer's copies: an asynchronous 4-byte report, no round trip)
-            if (static_cast<uint32_t>(h) == rank) mbar_arrive_expect_tx(&S.xfer[q], 4);
-            else st_async_signal(&S.mbox_x[q], &S.xfer[q], peer, 1u);
-          }
-          if (ok) pair_signal(rank, &S.v_full[q], &S.mbox_v[q], true, 4);   // quarter q landed here
-        }
-        if (!ok) break;
+      // ================================================================ V relay
+      // Forwards each landed V slice of this CTA to the even CTA's v_full barrier,
+      // which the PV issuer waits on.
+      int slot = 0;
+      uint32_t vph = 0;
+      for (int gv = 0; gv < nblk * kVSlices; ++gv) {
+        if (!mbar_wait(&S.v_loaded[slot], vph, p.status, ab)) break;
+        fence_proxy_async_smem();                            // cp.async writes -> tensor-core reads
+        pair_signal(rank, &S.v_full[slot], &S.mbox_v[slot], true, 4);
+        if (++slot == kVStages) { slot = 0; vph ^= 1; }
       }
-      // after an abort, copies already issued may still be landing: hold the CTA briefly
-      if (*ab)
-        for (int i = 0; i < 100; ++i) __nanosleep(1000);
     } else if (rank == 0 && lane == 0) {
       // ================================================================ MMA issuers (even CTA)
-      // Warp 12 issues S = Q K^T block after block, warp 15 issues O += P V.  With
-      // one issuer for both, S of block j+2 queued behind PV of block j, which
-      // waits for that block's softmax and V rows: the S ring then stayed full of
-      // consumed-late chunks and the gathers stalled.  The tensor pipe executes
-      // both streams; they touch disjoint TMEM columns.
-      // Waits use the CTA-scope try_wait, as 2-SM tensor-core pipelines do for the
-      // leader's stage barriers: a cluster-scope acquire on every stage cost about
-      // 0.35 us each and throttled MMA issue.
-      const uint32_t id_s = instr_desc(1, 1, false, false, 128, kBlk);   // bf16 x bf16, M=128 pair, N=128
+      // Warp 12 issues S = Q K^T block after block, warp 15 issues O += P V; the
+      // tensor pipe executes both streams, which touch disjoint TMEM columns.
+      // Waits use the CTA-scope try_wait, as 2-SM tensor-core pipelines do for
+      // the leader's stage barriers.  Descriptors are built once; a step inside a
+      // tile adds to the 14-bit start-address field (16-byte units).
+      const uint32_t id_s = instr_desc(1, 1, false, false, 128, kBlk);   // bf16 x bf16, M=128 pair, N=256
       const uint32_t id_pv = instr_desc(1, 1, false, true, 128, 256);    // B (V) MN-major, N=256
       bool ok = warp == 12 ? mbar_wait(&S.q_ready, 0, p.status, ab) : true;
-      // Descriptors are built once; a step inside a tile adds to the 14-bit
-      // start-address field (16-byte units).  Each ring holds exactly one block,
-      // so chunk c of every block sits in slot c and is in its (block)-th phase.
-      static_assert(kSStages == kDChunks, "one block per ring");
       const uint64_t qd0 = smem_desc_sw128(smem_u32(S.q[0]), 16, 1024);
       const uint64_t sd0 = smem_desc_sw128(smem_u32(S.s_ring[0]), 16, 1024);
       const uint64_t pd0 = smem_desc_sw128(smem_u32(S.p[0]), 16, 1024);
-      const uint64_t vd0 = smem_desc_sw128(smem_u32(S.vbuf[0]), kBlk * 128, 1024);
-      auto issue_s = [&](int j) -> bool {
-        const int sb = j & 1;
-        if (!mbar_wait(&S.s_free[sb], ((j >> 1) & 1) ^ 1, p.status, ab)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + kSCol + sb * 64;
-#pragma unroll
-        for (int ci = 0; ci < kDChunks; ++ci) {
-          const int dc = chunk_at(ci);
-          if (!mbar_wait(&S.s_full[dc], j & 1, p.status, ab)) return false;
+      const uint64_t vd0 = smem_desc_sw128(smem_u32(S.v_ring[0][0]), kVRows * 128, 1024);
+      if (ok && warp == 12) {
+        int slot = 0;
+        uint32_t sph = 0;
+        for (int j = 0; j < nblk && ok; ++j) {
+          const int sb = j & 1;
+          if (!mbar_wait(&S.s_free[sb], ((j >> 1) & 1) ^ 1, p.status, ab)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t d = tmem + kSCol + sb * 128;
+          for (int ci = 0; ci < kDChunks; ++ci) {
+            const int dc = chunk_at(ci);
+            if (!mbar_wait(&S.s_full[slot], sph, p.status, ab)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_bf16_pair(d, qd0 + static_cast<uint64_t>(dc * (kHalf * 128 / 16) + kk * 2),
-                           sd0 + static_cast<uint64_t>(dc * (kHalf * 128 / 16) + kk * 2), id_s, (ci | kk) != 0 ? 1u : 0u);
-          umma_commit_pair(&S.s_empty[dc], 0x3);
-        }
-        umma_commit_pair(&S.s_ready[sb], 0x3);
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(&S.p_full, j & 1, p.status, ab)) return false;
-        tc_fence_after();
-        // value dims quarter by quarter (c = V-buffer groups 2c, 2c+1): the
-        // quarter's tiles are released for the next block's copies as soon as its
-        // 8 MMAs completed, while the other quarter is still being multiplied
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (!mbar_wait(&S.v_full[c], j & 1, p.status, ab)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < kBlk / 16; ++kk) {
-            const uint64_t pa = pd0 + static_cast<uint64_t>((kk >> 2) * (kHalf * 128 / 16) + (kk & 3) * 2);
-            umma_bf16_pair(tmem + kOCol + c * 128, pa,
-                           vd0 + static_cast<uint64_t>(kk * (16 * 128 / 16) + c * (2 * kBlk * 128 / 16)), id_pv,
-                           (j | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_pair(d, qd0 + static_cast<uint64_t>(dc * (kHeads * 128 / 16) + kk * 2),
+                             sd0 + static_cast<uint64_t>(slot * (kRows * 128 / 16) + kk * 2), id_s,
+                             (ci | kk) != 0 ? 1u : 0u);
+            umma_commit_pair(&S.s_empty[slot], 0x3);
+            if (++slot == kSStages) { slot = 0; sph ^= 1; }
           }
-          umma_commit_pair(&S.v_empty[c], 0x3);
+          if (!ok) break;
+          umma_commit_pair(&S.s_ready[sb], 0x3);
         }
-        umma_commit_pair(&S.p_empty, 0x3);
-        return true;
-      };
-      if (ok) {
-        if (warp == 12) {
-          for (int j = 0; j < nblk && ok; ++j) ok = issue_s(j);
-        } else {
-          for (int j = 0; j < nblk && ok; ++j) ok = issue_pv(j);
+      } else if (ok) {
+        int slot = 0;
+        uint32_t vph = 0;
+        for (int j = 0; j < nblk && ok; ++j) {
+          if (!mbar_wait(&S.p_full, j & 1, p.status, ab)) { ok = false; break; }
+          tc_fence_after();
+          // slice by slice: each V slot's four MMAs (two 16-row K steps x two
+          // halves of the value dims) release it for the gathers of a later slice
+          for (int vs = 0; vs < kVSlices; ++vs) {
+            if (!mbar_wait(&S.v_full[slot], vph, p.status, ab)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+              const int ks = vs * 2 + k2;                      // 16-row K step of the block
+              const uint64_t pa = pd0 + static_cast<uint64_t>((ks >> 2) * (kHeads * 128 / 16) + (ks & 3) * 2);
+#pragma unroll
+              for (int c = 0; c < 2; ++c)
+                umma_bf16_pair(tmem + kOCol + c * 128, pa,
+                               vd0 + static_cast<uint64_t>(slot * (4 * kVRows * 128 / 16) + c * (2 * kVRows * 128 / 16) +
+                                                           k2 * (16 * 128 / 16)),
+                               id_pv, (j | ks) != 0 ? 1u : 0u);
+            }
+            umma_commit_pair(&S.v_empty[slot], 0x3);
+            if (++slot == kVStages) { slot = 0; vph ^= 1; }
+          }
+          if (!ok) break;
+          umma_commit_pair(&S.p_empty, 0x3);
         }
       }
       umma_commit_pair(&S.done, 0x1);                       // drain: this issuer's MMAs completed

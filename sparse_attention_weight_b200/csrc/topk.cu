@@ -27,6 +27,8 @@ constexpr int kThreads = 512;
 constexpr int kPer = 4;
 constexpr int kStep = kThreads * kPer;   // elements per block step
 constexpr int kCacheMax = 32768;         // keys cached in shared memory at most (128 KB)
+constexpr int kClusterMinLen = 8192;     // rows at least this long may share a cluster of CTAs
+constexpr int kClusterSegMax = 20480;    // keys cached per CTA of a cluster (80 KB: two CTAs per SM)
 
 __device__ __forceinline__ uint32_t order_key(float x) {
   uint32_t b = __float_as_uint(x);
@@ -64,6 +66,23 @@ __device__ __forceinline__ void load_keys(const Ctx& c, int i, bool from_cache, 
   }
   if (fill_cache && i < c.n) {
     *reinterpret_cast<uint4*>(c.cache + i) = make_uint4(k[0], k[1], k[2], k[3]);
+  }
+}
+
+// Adds each lane's bin (lanes with `in` set) to a shared-memory histogram.  A
+// warp with no lane in skips (most warps, in the passes that filter on a
+// prefix); a warp whose lanes all hold the same bin makes one atomic (ties,
+// constant rows); otherwise every lane adds its own.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool in, int lane) {
+  const uint32_t inmask = __ballot_sync(0xffffffffu, in);
+  if (inmask == 0) return;
+  const int leader = __ffs(inmask) - 1;
+  const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
+  const uint32_t same = __ballot_sync(0xffffffffu, in && bin == b0);
+  if (same == inmask) {
+    if (lane == leader) atomicAdd(&hist[b0], static_cast<uint32_t>(__popc(inmask)));
+  } else if (in) {
+    atomicAdd(&hist[bin], 1u);
   }
 }
 
@@ -107,9 +126,7 @@ __device__ void hist_pass(const Ctx& c, bool from_cache, bool fill_cache, uint32
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       const bool in = valid[u] && (fshift >= 32 || (k[u] >> fshift) == prefix);
-      const uint32_t bin = in ? ((k[u] >> shift) & mask) : 0xffffffffu;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+      hist_add(hist, (k[u] >> shift) & mask, in, lane);
     }
   }
 }
@@ -266,10 +283,9 @@ __device__ void hist_list(const uint32_t* keys, int m, uint32_t* hist, int shift
   const uint32_t mask = (1u << bits) - 1u;
   for (int base = 0; base < m; base += kThreads) {
     const int i = base + threadIdx.x;
-    const bool in = i < m && (keys[i < m ? i : 0] >> fshift) == prefix;
-    const uint32_t bin = in ? ((keys[i] >> shift) & mask) : 0xffffffffu;
-    const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-    if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
+    const uint32_t key = keys[i < m ? i : 0];
+    const bool in = i < m && (key >> fshift) == prefix;
+    hist_add(hist, (key >> shift) & mask, in, lane);
   }
 }
 
@@ -388,6 +404,224 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(TopkParams p) {
   }
 }
 
+// ---------------------------------------------------------------- few long rows: a cluster per row
+// When the rows are few (decode), one CTA per row leaves most SMs idle.  Here a
+// cluster of C CTAs (2, 4 or 8) shares a row: CTA r caches the keys of segment r
+// (consecutive indices) in its shared memory.  Each radix pass (11, 11 and 10
+// key bits) histograms the CTA's segment locally, then adds the non-zero bins
+// into every CTA's copy of the cluster histogram (remote reductions through
+// distributed shared memory, which need no round trip); after one cluster
+// barrier every CTA finds the same threshold bin in its own copy.  The output
+// pass writes each CTA's selected keys at the offset given by the selections of
+// the segments before it, so the result is in index order with ties going to
+// the lower index, as in the single-CTA kernels.  The row is read from memory
+// once; five cluster barriers in all.
+__device__ __forceinline__ uint32_t cl_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cl_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cl_map(const void* p, uint32_t cta) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(cta));
+  return r;
+}
+__device__ __forceinline__ void red_add_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+struct ClusterShared {
+  uint32_t local[2048];          // this CTA's histogram of the current pass
+  uint32_t global[2][2048];      // the cluster's histogram (passes alternate buffers)
+  uint32_t scratch[32];
+  uint32_t sel[2];
+  uint32_t cnt_gt[8], cnt_eq[8]; // per-CTA counts of keys above / equal to the threshold
+};
+
+// Adds this CTA's histogram (nbins bins) into every CTA's `global` buffer.
+__device__ __forceinline__ void cl_push(const ClusterShared& S, uint32_t* dst, int nbins, uint32_t C) {
+  for (int b = threadIdx.x; b < nbins; b += kThreads) {
+    const uint32_t v = S.local[b];
+    if (v == 0) continue;
+    for (uint32_t c = 0; c < C; ++c) red_add_cluster(cl_map(dst + b, c), v);
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, int seg_cap) {
+  extern __shared__ __align__(16) uint32_t tk_smem[];
+  ClusterShared& S = *reinterpret_cast<ClusterShared*>(tk_smem);
+  uint32_t* cache = tk_smem + (sizeof(ClusterShared) + 15) / 16 * 4;   // seg_cap keys
+  const uint32_t C = cl_size(), r = cl_rank();
+  const int t = blockIdx.x / static_cast<int>(C);
+  const int k = p.k;
+  const int lane = threadIdx.x & 31;
+  int32_t* out = p.idx + static_cast<int64_t>(t) * k;
+  // row length (identical in every CTA of the cluster, so all take the same branches)
+  int n = -1;
+  {
+    const int seq = p.q_seq[t];
+    if (seq >= 0 && seq < p.num_seqs) {
+      const int len = p.kv_len[seq];
+      const int pos = p.q_pos[t];
+      if (len >= 0 && len <= p.max_kv_len && pos >= 0 && pos < len) n = pos + 1;
+    }
+  }
+  if (n < 0 || n <= k) {                                   // every CTA writes its share of the row
+    if (n < 0 && r == 0 && threadIdx.x == 0) set_status(p.status, DSA_DEV_BAD_QUERY);
+    for (int j = static_cast<int>(r) * kThreads + threadIdx.x; j < k; j += static_cast<int>(C) * kThreads)
+      out[j] = (j < n) ? j : -1;
+    return;
+  }
+  const int seg = ((n + static_cast<int>(C) - 1) / static_cast<int>(C) + kPer - 1) / kPer * kPer;
+  if (seg > seg_cap) {                                     // cannot happen with the host's sizing
+    if (r == 0 && threadIdx.x == 0) set_status(p.status, DSA_DEV_INTERNAL);
+    for (int j = static_cast<int>(r) * kThreads + threadIdx.x; j < k; j += static_cast<int>(C) * kThreads) out[j] = -1;
+    return;
+  }
+  const int lo = min(n, static_cast<int>(r) * seg);
+  const int m = min(n, lo + seg) - lo;                     // keys of this CTA's segment
+  const float* row = p.scores + static_cast<int64_t>(t) * p.ld + lo;
+
+  for (int b = threadIdx.x; b < 2048; b += kThreads) {
+    S.local[b] = 0;
+    S.global[0][b] = 0;
+    S.global[1][b] = 0;
+  }
+  __syncthreads();
+  cl_sync();                                               // every copy is cleared before any reduction
+
+  // pass 1: cache the segment's keys and histogram bits 31..21; four 16-byte
+  // loads per thread in flight
+  constexpr int kUnroll = 4;
+  for (int base = 0; base < m; base += kStep * kUnroll) {
+    uint32_t kk[kUnroll][kPer];
+#pragma unroll
+    for (int w = 0; w < kUnroll; ++w) {
+      const int i = base + w * kStep + threadIdx.x * kPer;
+      if (i + kPer <= m) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(row + i));   // lo and ld are multiples of 4
+        kk[w][0] = order_key(f.x); kk[w][1] = order_key(f.y); kk[w][2] = order_key(f.z); kk[w][3] = order_key(f.w);
+      } else {
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) kk[w][u] = (i + u) < m ? order_key(__ldg(row + i + u)) : 0u;
+      }
+    }
+#pragma unroll
+    for (int w = 0; w < kUnroll; ++w) {
+      const int i = base + w * kStep + threadIdx.x * kPer;
+      if (i < m) *reinterpret_cast<uint4*>(cache + i) = make_uint4(kk[w][0], kk[w][1], kk[w][2], kk[w][3]);
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        hist_add(S.local, kk[w][u] >> 21, (i + u) < m, lane);
+      }
+    }
+  }
+  __syncthreads();
+  cl_push(S, S.global[0], 2048, C);
+  cl_sync();                                               // the cluster's histogram is complete everywhere
+  find_bin(S.global[0], 2048, static_cast<uint32_t>(k), S.scratch, &S.sel[0], &S.sel[1]);
+  const uint32_t b1 = S.sel[0], r1 = S.sel[1];
+  __syncthreads();
+
+  // pass 2: bits 20..10 of the keys with the pass-1 prefix (global[1] was cleared at the start)
+  for (int b = threadIdx.x; b < 2048; b += kThreads) {
+    S.local[b] = 0;
+    S.global[0][b] = 0;                                    // read above; peers write it again only after the next barrier
+  }
+  __syncthreads();
+  const Ctx cc{nullptr, cache, m};
+  hist_pass(cc, true, false, S.local, 10, 11, 21, b1);
+  __syncthreads();
+  cl_push(S, S.global[1], 2048, C);
+  cl_sync();
+  find_bin(S.global[1], 2048, r1, S.scratch, &S.sel[0], &S.sel[1]);
+  const uint32_t b2 = S.sel[0], r2 = S.sel[1];
+  __syncthreads();
+
+  // pass 3: bits 9..0
+  const uint32_t pre2 = (b1 << 11) | b2;
+  for (int b = threadIdx.x; b < 2048; b += kThreads) S.local[b] = 0;
+  __syncthreads();
+  hist_pass(cc, true, false, S.local, 0, 10, 10, pre2);
+  __syncthreads();
+  cl_push(S, S.global[0], 1024, C);
+  cl_sync();
+  find_bin(S.global[0], 1024, r2, S.scratch, &S.sel[0], &S.sel[1]);
+  const uint32_t tau = (pre2 << 10) | S.sel[0];            // the k-th largest key
+  const uint32_t need = S.sel[1];                          // its copies to take, lowest indices first
+  __syncthreads();
+
+  // counts above / equal to tau of every segment -> offsets of this segment's output
+  {
+    uint32_t cgt = 0, ceq = 0;
+    for (int i = threadIdx.x; i < m; i += kThreads) {
+      const uint32_t key = cache[i];
+      cgt += key > tau ? 1u : 0u;
+      ceq += key == tau ? 1u : 0u;
+    }
+    uint32_t tgt, teq;
+    block_scan(cgt, S.scratch, &tgt);
+    block_scan(ceq, S.scratch, &teq);
+    if (threadIdx.x < static_cast<int>(C)) {
+      st_cluster(cl_map(&S.cnt_gt[r], threadIdx.x), tgt);
+      st_cluster(cl_map(&S.cnt_eq[r], threadIdx.x), teq);
+    }
+  }
+  cl_sync();                                               // last access to another CTA's memory
+  uint32_t gt_base = 0, eq_base = 0;
+  for (uint32_t c = 0; c < r; ++c) { gt_base += S.cnt_gt[c]; eq_base += S.cnt_eq[c]; }
+
+  // output pass over the cached segment, index order (global index = lo + i)
+  for (int base = 0; base < m; base += kStep) {
+    const int i = base + threadIdx.x * kPer;
+    uint32_t kk[kPer];
+    bool valid[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      valid[u] = i + u < m;
+      kk[u] = valid[u] ? cache[i + u] : 0u;
+    }
+    uint32_t cgt = 0, ceq = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      cgt += (valid[u] && kk[u] > tau) ? 1u : 0u;
+      ceq += (valid[u] && kk[u] == tau) ? 1u : 0u;
+    }
+    const uint32_t packed = cgt | (ceq << 16);
+    uint32_t total;
+    const uint32_t incl = block_scan(packed, S.scratch, &total);
+    const uint32_t excl = incl - packed;
+    uint32_t gt_before = gt_base + (excl & 0xffffu);
+    uint32_t eq_before = eq_base + (excl >> 16);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (!valid[u]) continue;
+      if (kk[u] > tau) {
+        const uint32_t slot = gt_before + min(eq_before, need);
+        if (slot < static_cast<uint32_t>(k)) out[slot] = lo + i + u;
+        ++gt_before;
+      } else if (kk[u] == tau) {
+        const uint32_t slot = gt_before + eq_before;
+        if (eq_before < need && slot < static_cast<uint32_t>(k)) out[slot] = lo + i + u;
+        ++eq_before;
+      }
+    }
+    gt_base += total & 0xffffu;
+    eq_base += total >> 16;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
@@ -397,9 +631,45 @@ cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
                                                   cudaSuccess)
     sms = 148;
-  // Long rows.  With few rows (at most two per SM: decode) each CTA has an SM to
-  // itself and reading the row twice instead of four times wins; with many rows
-  // the streaming kernel, four CTAs per SM, keeps more loads in flight.
+  // A cluster of C CTAs per row (C in 2, 4, 8), each caching one segment, when
+  // the rows are too long for one CTA's cache (C = the fewest CTAs whose
+  // segments fit) or too few to fill the SMs (C = the most CTAs that keep the
+  // grid within two per SM).
+  if (p.max_kv_len >= kClusterMinLen) {
+    // segment cache, rounded up to whole block steps: the passes over it read in steps of kStep keys
+    auto seg_of = [&](int c) { return (((p.max_kv_len + c - 1) / c + kStep - 1) / kStep) * kStep; };
+    int c_fit = 1;
+    while (c_fit <= 8 && seg_of(c_fit) > kClusterSegMax) c_fit <<= 1;
+    int c_par = 8;
+    while (c_par > 1 && T * c_par > 2 * sms) c_par >>= 1;
+    const int C = c_fit > c_par ? c_fit : c_par;
+    if (C >= 2 && C <= 8) {
+      const int seg_cap = seg_of(C);
+      const size_t smem = (sizeof(ClusterShared) + 15) / 16 * 16 + static_cast<size_t>(seg_cap) * sizeof(uint32_t);
+      cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(T * C));
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = smem;
+      cfg.stream = stream;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, p, seg_cap);
+      if (e == cudaSuccess) count_launches(1);
+      return e;
+    }
+  }
+  // Rows longer than eight segments.  With few rows (at most two per SM) each CTA
+  // has an SM to itself and reading the row twice instead of four times wins;
+  // with many rows the streaming kernel, four CTAs per SM, keeps more loads in
+  // flight.
   if (cache_elems > kCacheMax && T <= 2 * sms) {      // two reads and a candidate list
     const size_t smem = ((1 << kHiBits) + 64 + 2 * kListCap) * sizeof(uint32_t);
     cudaError_t e = cudaFuncSetAttribute(topk_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

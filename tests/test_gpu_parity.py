@@ -137,20 +137,42 @@ def test_topk_adversarial_rows(cuda_device):
 
 
 def test_topk_long_rows_from_l2(cuda_device):
-    """Rows longer than the shared-memory cache: two reads and a candidate list,
-    and the streaming fallback when the threshold's bin overflows the list."""
+    """Rows longer than a cluster's eight segment caches (> 163840 keys): two reads
+    and a candidate list for few rows, with the streaming fallback when the
+    threshold's bin overflows the list; the streaming kernel for many rows."""
     rng = np.random.default_rng(12)
-    rows = [rng.standard_normal(40000).astype(np.float32),
-            np.round(rng.standard_normal(131072), 2).astype(np.float32),
-            rng.standard_normal(33000).astype(np.float32),
-            np.zeros(40000, np.float32),                                     # all tied: fallback
-            rng.integers(-3, 4, size=50000).astype(np.float32),              # 7 values: fallback
-            np.concatenate([np.full(3000, 2.0), rng.standard_normal(60000) - 10.0]).astype(np.float32),
+    rows = [rng.standard_normal(170000).astype(np.float32),
+            np.round(rng.standard_normal(180000), 2).astype(np.float32),
+            np.zeros(170000, np.float32),                                    # all tied: fallback
+            rng.integers(-3, 4, size=170000).astype(np.float32),             # 7 values: fallback
+            np.concatenate([np.full(3000, 2.0), rng.standard_normal(170000) - 10.0]).astype(np.float32),
             rng.standard_normal(1500).astype(np.float32)]                    # n <= k in a long launch
     _topk_case(cuda_device, rows, 2048)
-    # many long rows (more than two per SM): the streaming kernel reads them from L2
-    many = [np.round(rng.standard_normal(int(n)), 3).astype(np.float32) for n in rng.integers(33000, 40000, 320)]
+    # many very long rows (more than two per SM): the streaming kernel reads them from L2
+    many = [np.round(rng.standard_normal(int(n)), 3).astype(np.float32) for n in rng.integers(164000, 166000, 300)]
     _topk_case(cuda_device, many, 2048)
+    # many long rows that fit eight segment caches: one cluster per row
+    many = [np.round(rng.standard_normal(int(n)), 3).astype(np.float32) for n in rng.integers(33000, 70000, 320)]
+    _topk_case(cuda_device, many, 2048)
+
+
+def test_topk_rows_shared_by_a_cluster(cuda_device):
+    """Few long rows: a cluster of CTAs per row (8, 4 or 2 of them, by the number of
+    rows), each caching one segment; ties across segment boundaries go to the lower
+    index, and rows with n <= k or mass ties take the same cluster path."""
+    rng = np.random.default_rng(13)
+    k = 2048
+    base = [np.round(rng.standard_normal(20000), 1).astype(np.float32),          # ties across segments
+            np.zeros(16384, np.float32),                                         # all equal
+            np.concatenate([rng.standard_normal(9000), np.full(9000, 5.0)]).astype(np.float32),
+            rng.standard_normal(8193).astype(np.float32),
+            rng.standard_normal(2000).astype(np.float32),                        # n <= k
+            np.where(rng.random(12000) < 0.5, -0.0, 0.0).astype(np.float32)]
+    for T in (6, 40, 100):              # clusters of 8, 4 (6 rows -> 8; 40 -> 4...) and 2 CTAs
+        rows = [base[t % len(base)] if t < len(base) else rng.standard_normal(int(rng.integers(8192, 30000)))
+                .astype(np.float32) for t in range(T)]
+        _topk_case(cuda_device, rows, k)
+    _topk_case(cuda_device, base[:3], 100)
 
 # ----------------------------------------------------------------------------- sparse MLA
 
