@@ -81,11 +81,12 @@ struct MlaSmem {
   uint64_t s_full[kSStages], s_empty[kSStages], s_loaded[kSStages];
   uint64_t v_full[kVStages], v_empty[kVStages], v_loaded[kVStages];
   uint64_t s_ready[2], s_free[2];
-  uint64_t p_full, p_empty;
+  uint64_t p_full[2], p_empty[2];            // per half of P: rows 0..127 (chunks 0-1), 128..255 (chunks 2-3)
   uint64_t mx_bar[2], l_bar;
+  uint64_t o_done[2];                         // O lanes of warp 2+i rescaled (local, for warp i)
   uint64_t done;
   // mailboxes of the peer CTA's asynchronous signals (contents unused)
-  uint32_t mbox_q, mbox_s[kSStages], mbox_v[kVStages], mbox_sfree[2][4], mbox_pfull[4];
+  uint32_t mbox_q, mbox_s[kSStages], mbox_v[kVStages], mbox_sfree[2][4], mbox_pfull[2][2];
   uint32_t tmem_base;
   int last_used[8];                          // per prologue warp: last usable entry, -1 if none
   int abort_flag;
@@ -174,9 +175,9 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 4); mbar_init(&S.mx_bar[i], 128);
     }
-    mbar_init(&S.p_full, 4);
-    mbar_init(&S.p_empty, 1);
+    for (int h = 0; h < 2; ++h) { mbar_init(&S.p_full[h], 2); mbar_init(&S.p_empty[h], 1); }
     mbar_init(&S.l_bar, 128);
+    mbar_init(&S.o_done[0], 1); mbar_init(&S.o_done[1], 1);
     mbar_init(&S.done, 2);                      // one drain commit per MMA issuer
     S.abort_flag = 0;
     if (smem_u32(smem_raw) & 1023u) {           // the swizzled tiles need 1024-byte alignment
@@ -240,6 +241,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       const int half = tid >> 6;
       const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
       float m_ref = -INFINITY, l = 0.f;
+      uint32_t n_rescaled = 0;                               // blocks j > 0 that rescaled O (this warp)
       for (int j = 0; j < nblk; ++j) {
         const int sb = j & 1;
         const uint32_t sph = (j >> 1) & 1;
@@ -272,11 +274,45 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         // subtract 0 instead, so that each p is 2^-inf = 0 (never -inf - -inf)
         const float msub = m_new == -INFINITY ? 0.f : m_new;
         const float alpha = rescale ? ex2_approx(m_ref - m_new) : 1.f;   // m_ref = -inf -> 0
-        // P buffer and O are free once PV of the previous block completed
+        const bool rs_any = __any_sync(0xffffffffu, rescale);   // warp-uniform (TMEM ld/st are warp-collective)
+        const bool rs_wait = j > 0 && rs_any;
+        // pass 2: P = 2^(x - m) in bf16, held in registers (64 packed pairs) so
+        // that the S buffer is released before the P buffer is free; the
+        // denominator sums the same bf16 values that the PV MMA multiplies V by
+        float psum = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {                         // 16 columns at a time
+          uint32_t sr[16];
+          tmem_ld16(sbase + c * 16, sr);
+          const uint32_t vmc = valid_word(c >> 1) >> ((c & 1) * 16);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 16; u += 2) {
+            const float x0 = ((vmc >> u) & 1u) ? __uint_as_float(sr[u]) * p.sm_scale_log2 : -INFINITY;
+            const float x1 = ((vmc >> (u + 1)) & 1u) ? __uint_as_float(sr[u + 1]) * p.sm_scale_log2 : -INFINITY;
+            const uint32_t pp = pack_bf16(ex2_approx(x0 - msub), ex2_approx(x1 - msub));
+            psum += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
+            pk[c * 8 + (u >> 1)] = pp;
+          }
+        }
+        l = l * alpha + psum;
+        m_ref = m_new;
+        // S buffer sb has been read: the S MMAs of block j+2 may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) pair_signal(rank, &S.s_free[sb], &S.mbox_sfree[sb][warp], warp == 0, 16);
+        // This thread's half of P (rows 128*half ..) is free once the PV MMAs of
+        // block j-1 on it completed: the PV consumes rows 0..127 first, so half 0
+        // stores while the PV still multiplies the other half.  O may be rescaled
+        // only once the whole PV of block j-1 completed.  Warps w and w+2 hold the
+        // same heads, so they take the same rescale decision; the PV of block j
+        // starts on half 0's signal, so warp w then also waits for warp w+2 to
+        // have rescaled its O lanes before it signals.
         if (j > 0) {
-          if (!warp_wait(&S.p_empty, (j - 1) & 1, p.status, ab, false)) break;
+          if (!warp_wait(&S.p_empty[(half == 1 || rs_any) ? 1 : 0], (j - 1) & 1, p.status, ab, false)) break;
           tc_fence_after();
-          if (__any_sync(0xffffffffu, rescale)) {   // TMEM ld/st are warp-collective
+          if (rs_any) {
 #pragma unroll 1
             for (int c = 0; c < 16; ++c) {
               uint32_t o[16];
@@ -288,48 +324,41 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
               tmem_st16(a, o);
             }
             tmem_st_wait();
+            if (half == 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&S.o_done[warp & 1]);
+            }
           }
         }
-        m_ref = m_new;
-        // pass 2: P = 2^(x - m) in bf16, written as P row hl of K chunks 2*half and
-        // 2*half+1 (rows 128*half .. +127 of the block), 128B-swizzled; the
-        // denominator sums the same bf16 values that the PV MMA multiplies V by
-        float psum = 0.f;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sr[32];
-          tmem_ld32(sbase + c * 32, sr);
-          const uint32_t vmc = valid_word(c);
-          tmem_ld_wait();
-          uint32_t pk[16];
+        // P row hl of K chunks 2*half and 2*half+1 (rows 128*half .. +127 of the
+        // block), 128B-swizzled
 #pragma unroll
-          for (int u = 0; u < 32; u += 2) {
-            const float x0 = ((vmc >> u) & 1u) ? __uint_as_float(sr[u]) * p.sm_scale_log2 : -INFINITY;
-            const float x1 = ((vmc >> (u + 1)) & 1u) ? __uint_as_float(sr[u + 1]) * p.sm_scale_log2 : -INFINITY;
-            const uint32_t pp = pack_bf16(ex2_approx(x0 - msub), ex2_approx(x1 - msub));
-            psum += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
-            pk[u >> 1] = pp;
-          }
+        for (int c = 0; c < 4; ++c) {
           uint8_t* prow = S.p[half * 2 + (c >> 1)] + hl * 128;
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const int c16 = (c & 1) * 4 + q4;                // 16-byte chunk of the 128-byte row
             *reinterpret_cast<uint4*>(prow + ((c16 ^ (hl & 7)) << 4)) =
-                make_uint4(pk[q4 * 4 + 0], pk[q4 * 4 + 1], pk[q4 * 4 + 2], pk[q4 * 4 + 3]);
+                make_uint4(pk[c * 16 + q4 * 4 + 0], pk[c * 16 + q4 * 4 + 1], pk[c * 16 + q4 * 4 + 2],
+                           pk[c * 16 + q4 * 4 + 3]);
           }
         }
-        l = l * alpha + psum;
-        // S buffer sb has been read: the S MMAs of block j+2 may overwrite it
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) pair_signal(rank, &S.s_free[sb], &S.mbox_sfree[sb][warp], warp == 0, 16);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) pair_signal(rank, &S.p_full, &S.mbox_pfull[warp], warp == 0, 16);
+        if (half == 0 && rs_wait) {
+          if (!warp_wait(&S.o_done[warp & 1], n_rescaled & 1, p.status, ab, false)) break;
+          tc_fence_after();
+          tc_fence_before();
+        }
+        if (rs_wait) ++n_rescaled;
+        // per half: warps 2*half, 2*half+1 of both CTAs (the even one's first warp
+        // carries the odd CTA's 8 bytes)
+        if (lane == 0) pair_signal(rank, &S.p_full[half], &S.mbox_pfull[half][warp & 1], (warp & 1) == 0, 8);
       }
       // ---- epilogue: wait for the last PV, combine the two row halves, write out
       bool ok = !*ab;
-      if (ok) ok = warp_wait(&S.p_empty, (nblk - 1) & 1, p.status, ab, false);
+      if (ok) ok = warp_wait(&S.p_empty[1], (nblk - 1) & 1, p.status, ab, false);
       if (ok) {
         tc_fence_after();
         S.lsum[tid] = l;
@@ -534,11 +563,18 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         int slot = 0;
         uint32_t vph = 0;
         for (int j = 0; j < nblk && ok; ++j) {
-          if (!mbar_wait(&S.p_full, j & 1, p.status, ab)) { ok = false; break; }
+          if (!mbar_wait(&S.p_full[0], j & 1, p.status, ab)) { ok = false; break; }
           tc_fence_after();
           // slice by slice: each V slot's four MMAs (two 16-row K steps x two
           // halves of the value dims) release it for the gathers of a later slice
           for (int vs = 0; vs < kVSlices; ++vs) {
+            if (vs == kVSlices / 2) {
+              // rows 0..127 of P consumed: half 0 of block j+1 may overwrite them;
+              // rows 128..255 must have been written by now
+              umma_commit_pair(&S.p_empty[0], 0x3);
+              if (!mbar_wait(&S.p_full[1], j & 1, p.status, ab)) { ok = false; break; }
+              tc_fence_after();
+            }
             if (!mbar_wait(&S.v_full[slot], vph, p.status, ab)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
@@ -556,7 +592,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
             if (++slot == kVStages) { slot = 0; vph ^= 1; }
           }
           if (!ok) break;
-          umma_commit_pair(&S.p_empty, 0x3);
+          umma_commit_pair(&S.p_empty[1], 0x3);
         }
       }
       umma_commit_pair(&S.done, 0x1);                       // drain: this issuer's MMAs completed
