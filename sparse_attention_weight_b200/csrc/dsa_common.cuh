@@ -353,6 +353,18 @@ __host__ __device__ __forceinline__ uint32_t sw128(uint32_t byte_off) {
   return byte_off ^ (((byte_off >> 7) & 7u) << 4);
 }
 
+// Register reallocation between warpgroups (all four warps of a warpgroup
+// execute the same instruction).  An increase waits until other warpgroups have
+// released enough of the registers the CTA was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ uint32_t elect_one_sync() {
   uint32_t pred = 0;
   asm volatile(
