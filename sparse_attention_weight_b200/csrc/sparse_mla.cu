@@ -76,10 +76,10 @@ constexpr int kBlk = 256;             // selected rows per block (pair)
 constexpr int kRows = 128;            // rows per CTA per block (S operand)
 constexpr int kHeads = 64;            // heads per CTA
 constexpr int kDChunks = DSA_D_QK / 64;   // 9 chunks of 64 dims
-constexpr int kSStages = 4;           // S ring: 16 KB slots (128 rows x 64 dims)
+constexpr int kSStages = 3;           // S ring: 16 KB slots (128 rows x 64 dims)
 constexpr int kVRows = 32;            // rows per V slice
 constexpr int kVSlices = kBlk / kVRows;   // 8 slices per block
-constexpr int kVStages = 3;           // V ring: 16 KB slots (32 rows x 256 value dims)
+constexpr int kVStages = 4;           // V ring: 16 KB slots (32 rows x 256 value dims)
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 constexpr uint32_t kSCol = 0;         // TMEM columns [0,256): two S buffers of 128
 constexpr uint32_t kOCol = 256;       // TMEM columns [256,512): O (2 x 128)
