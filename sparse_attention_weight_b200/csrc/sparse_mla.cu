@@ -18,14 +18,18 @@
 //                softmax warps), B = V rows of the block, each CTA holding 128
 //                of every 256 value dims (MN-major), N = 256; per CTA: 64 heads
 //                x 512 dims fp32 (256 TMEM columns).
-// A single tcgen05.mma takes longer to issue (about 58 ns) than a pair MMA of
-// 64 x 128 per SM takes to execute, so the block is 256 rows wide: every S
-// and PV instruction then moves 64 x 256 per SM, and a block needs 68 of them.
-// S is double buffered in TMEM, so the tensor core computes S of block j+1
-// while the softmax warps turn S of block j into P.  The softmax keeps a
-// reference maximum per head and rescales O (in TMEM) only when a block's
-// maximum exceeds it by more than 2^8, so P stays <= 256 and most blocks skip
-// the rescale.
+// A pair MMA with N = 128 takes about as long as one with N = 256 (measured
+// 35.5 vs 36.7 ns), so the block is 256 rows wide: every S and PV instruction
+// moves 64 x 256 per SM, and a block needs 68 of them.  S is double buffered in
+// TMEM, so the tensor core computes S of block j+1 while the softmax warps turn
+// S of block j into P.  The softmax keeps a reference maximum per head and
+// rescales O (in TMEM) only when a block's maximum exceeds it by more than 2^8,
+// so P stays <= 256 and most blocks skip the rescale.
+//
+// Persistent pairs: a pair walks the items (query, split) cid, cid + pairs, ...;
+// the rings and the per-block barriers count across items, so the next query's
+// index scan, gathers, Q load and first S MMAs overlap the current query's last
+// softmax, PV and output.
 //
 // Rows are gathered from L2 by index with 16-byte cp.async (8 lanes per 128-byte
 // row segment: coalesced) into 128-byte-swizzled tiles.  Two streaming rings
@@ -33,20 +37,23 @@
 // CTA's 128 rows (16 KB slots, refilled as soon as the S MMAs read them) and
 // the V ring holds 32-row slices of the block with the CTA's value dims (16 KB
 // slots, refilled as soon as the PV MMAs read them).  Each CTA thus reads the
-// value dims it multiplies straight from L2; no V data crosses the pair.
+// value dims it multiplies straight from L2; no V data crosses the pair.  The
+// gathers' shared-memory writes and the MMAs' operand reads share the SM's
+// shared-memory bandwidth (measured: gathers alone 73 B/clk, with back-to-back
+// MMAs 41 B/clk while the MMAs slow from 128 to 160 clk each).
 //
-// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-11 gathers of the
-// S ring, 12-19 gathers of the V ring, 20 TMEM owner and (in the even CTA)
-// issuer of the S MMAs, 21 Q load and S relay, 22 V relay, 23 (even CTA) issuer
-// of the PV MMAs.  Sixteen gather warps: one SM's 16-byte cp.async gathers from
-// L2 scale with the number of warps issuing them (about 27 B/clk with eight,
-// 42 with sixteen).  Signals from the odd CTA to the even CTA's barriers are
-// asynchronous 4-byte stores counted as transaction bytes (a thread-level
-// remote mbarrier arrive stalls its thread for a round trip).  Gather threads
-// never wait for their own copies: each arrives on a local stage barrier
-// through cp.async.mbarrier.arrive (hardware-tracked completion), and a relay
-// lane that has no copies in flight forwards the completed stage to the even
-// CTA's barrier, which the MMA issuer waits on.
+// Warps: 0-3 softmax / output (TMEM lane quadrants 0-3), 4-11 index scans and
+// gathers of the S ring, 12-19 gathers of the V ring, 20 TMEM owner, Q loads
+// (both CTAs) and (in the even CTA) issuer of the S MMAs, 21 S relay, 22 V
+// relay, 23 (even CTA) issuer of the PV MMAs.  Sixteen gather warps: one SM's
+// 16-byte cp.async gathers from L2 scale with the number of warps issuing them
+// (about 27 B/clk with eight, 42 with sixteen).  Signals from the odd CTA to
+// the even CTA's barriers are asynchronous 4-byte stores counted as transaction
+// bytes (a thread-level remote mbarrier arrive stalls its thread for a round
+// trip).  Gather threads never wait for their own copies: each arrives on a
+// local stage barrier through cp.async.mbarrier.arrive (hardware-tracked
+// completion), and a relay lane that has no copies in flight forwards the
+// completed stage to the even CTA's barrier, which the MMA issuer waits on.
 #include <cuda_bf16.h>
 
 #include "dsa_common.cuh"
