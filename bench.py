@@ -10,6 +10,8 @@ the line also carries, under "workloads", the other full-size workloads timed
 the same way in the same run:
   decode_b64        64 sequences, context U[4096, 32768], 1 query each;
   decode_128k_mtp2  16 sequences at context 131072, 2 queries each;
+  decode_b1_128k    1 sequence at context 131072, 1 query, paged cache
+                    (pages of 64 rows scattered over the cache pool);
   chunked_64k       a 65536-token prefill run as 16 calls of 4096 queries
                     against the growing cache (one step = all 16 calls).
 Inputs are seeded synthetic data resident in HBM when the timed region starts
@@ -57,6 +59,8 @@ D_QK, D_V, D_INDEX = 576, 512, 128
 # divided by its 2304 queries (the traffic is the queries in and the outputs out;
 # the gathered cache rows hit L2).  None while no capture describes the kernel.
 MLA_TRAFFIC_BYTES_PER_QUERY = (361.357568e6 + 258.470656e6) / 2304
+# Workloads run with a paged cache, and their page size (rows).
+PAGED = {"decode_b1_128k": 64}
 
 
 def mla_flop_per_pair(heads: int) -> int:
@@ -207,13 +211,14 @@ def algorithmic_pairs(q_pos: np.ndarray, k: int) -> tuple[int, int]:
 class Call:
     """Device buffers and workspaces of one call (one batch) of the path."""
 
-    def __init__(self, wl, bh, dev: dict, device, out=None, lse=None, kv_rows=None, scores=None, idx=None):
+    def __init__(self, wl, bh, dev: dict, device, out=None, lse=None, kv_rows=None, scores=None, idx=None,
+                 page_size=0, page_table=None):
         import torch
 
         from sparse_attention_weight_b200 import binding as B
         self.B = B
         self.wl, self.bh, self.dev = wl, bh, dev
-        self.db = B.DeviceBatch.from_host(bh, device, kv_rows=kv_rows)
+        self.db = B.DeviceBatch.from_host(bh, device, kv_rows=kv_rows, page_size=page_size, page_table=page_table)
         T = bh.num_q
         self.T = T
         self.ld = (bh.max_kv_len + 3) // 4 * 4
@@ -366,6 +371,17 @@ def device_calls(wl, device, seed):
         return calls
     bh = inputs.make_batch(wl, seed)
     dev = {**inputs.device_query_tensors(wl, bh, device, seed), **inputs.device_cache_tensors(wl, bh, device, seed)}
+    if wl.name in PAGED:
+        # the same rows scattered into pages of the cache pool
+        ps = PAGED[wl.name]
+        table, src = inputs.paged_layout(bh, ps, seed)
+        src_t = torch.as_tensor(src, device=device)
+        used = src_t >= 0
+        for name in ("k_idx", "kv"):
+            pool = torch.zeros((src.size, dev[name].shape[1]), dtype=dev[name].dtype, device=device)
+            pool[used] = dev[name][src_t[used]]
+            dev[name] = pool
+        return [Call(wl, bh, dev, device, kv_rows=src.size, page_size=ps, page_table=table)]
     return [Call(wl, bh, dev, device)]
 
 
@@ -396,6 +412,7 @@ def config_of(wl, args) -> dict:
             "seq_len": wl.seq_len or None, "batch": wl.batch or None,
             "ctx": [wl.ctx_min, wl.ctx_max] if decode else None, "q_per_seq": wl.q_per_seq or None,
             "chunk": wl.chunk or None, "l2": "flushed before every timed step (512 MB write)",
+            "kv_layout": f"paged, {PAGED[wl.name]}-row pages" if wl.name in PAGED else "contiguous per sequence",
             "parallelism": f"dp{args.gpus}" if args.gpus > 1 else "single"}
 
 
@@ -598,7 +615,7 @@ def main():
     # ---- the other full-size workloads, in the same run
     if not args.no_extra and not args.seq_len and not args.batch:
         line["workloads"] = {}
-        for name in ("decode_b64", "decode_128k_mtp2", "chunked_64k"):
+        for name in ("decode_b64", "decode_128k_mtp2", "decode_b1_128k", "chunked_64k"):
             if name != wl.name:
                 line["workloads"][name] = sub_record(WORKLOADS[name], args, rank, world, device, peaks)
 

@@ -26,7 +26,11 @@
  *     status word at the start of the workspace `ws`; each call clears the word
  *     when it starts.  Read it with dsa_read_device_status.
  *   - Batches: sequence b owns the cache rows kv_offset[b] .. kv_offset[b] +
- *     kv_len[b] - 1 of k_idx and kv (rows of one sequence are contiguous).
+ *     kv_len[b] - 1 of k_idx and kv (rows of one sequence are contiguous), or,
+ *     with a paged layout (page_size > 0), key s of sequence b sits in cache row
+ *     page_table[b * pages_per_seq + s / page_size] * page_size + s % page_size
+ *     (the block-table layout of paged inference caches: a sequence's rows are
+ *     contiguous only within a page).  Both k_idx and kv use the same rows.
  *     Query t belongs to sequence q_seq[t] and sees its keys 0 .. q_pos[t]
  *     (n_t = q_pos[t] + 1 keys; causal and inclusive).  Key and selection
  *     indices are local to the sequence.
@@ -41,7 +45,7 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 1
+#define DSA_ABI_VERSION 2
 
 /* Fixed widths of the method (one indexer key per token of 128 dims; latent 512
  * + RoPE 64; value = latent). */
@@ -75,6 +79,16 @@ typedef struct dsa_batch {
   const int32_t *kv_len;   /* (device) [B] cache rows of sequence b */
   const int32_t *q_seq;    /* (device) [T] sequence of query t */
   const int32_t *q_pos;    /* (device) [T] position of query t, 0 <= q_pos < kv_len */
+  /* Paged layout (ABI 2).  page_size = 0: contiguous rows from kv_offset (the
+   * fields below are ignored).  page_size > 0: a multiple of 64; kv_offset is
+   * ignored (may be NULL); page_table (device) int32 [B, pages_per_seq] holds the
+   * physical page of each page of a sequence, pages_per_seq * page_size >=
+   * max_kv_len; kv_rows is the number of physical rows (pages * page_size).  A
+   * page entry that points outside kv_rows raises DSA_DEV_BAD_INDEX and reads
+   * as zeros. */
+  int32_t page_size;
+  int32_t pages_per_seq;
+  const int32_t *page_table;
 } dsa_batch;
 
 /* Operation codes for dsa_workspace_size. */

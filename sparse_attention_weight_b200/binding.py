@@ -43,7 +43,8 @@ class DsaBatch(ctypes.Structure):
     _fields_ = [("num_seqs", ctypes.c_int32), ("num_q", ctypes.c_int32), ("max_kv_len", ctypes.c_int32),
                 ("max_q_per_seq", ctypes.c_int32), ("kv_rows", ctypes.c_int64),
                 ("kv_offset", ctypes.c_void_p), ("kv_len", ctypes.c_void_p), ("q_seq", ctypes.c_void_p),
-                ("q_pos", ctypes.c_void_p)]
+                ("q_pos", ctypes.c_void_p), ("page_size", ctypes.c_int32), ("pages_per_seq", ctypes.c_int32),
+                ("page_table", ctypes.c_void_p)]
 
 
 _lib = None
@@ -102,11 +103,15 @@ class DeviceBatch:
     q_seq: torch.Tensor
     q_pos: torch.Tensor
     struct: DsaBatch
+    page_table: torch.Tensor | None = None
 
     @classmethod
     def from_host(cls, b, device, kv_rows: int | None = None, max_kv_len: int | None = None,
-                  max_q_per_seq: int | None = None) -> "DeviceBatch":
-        """`b` has numpy kv_offset, kv_len, q_seq, q_pos (e.g. inputs.Batch)."""
+                  max_q_per_seq: int | None = None, page_size: int = 0,
+                  page_table=None) -> "DeviceBatch":
+        """`b` has numpy kv_offset, kv_len, q_seq, q_pos (e.g. inputs.Batch).  With
+        page_size > 0, `page_table` is an int32 array [B, pages_per_seq] of physical
+        pages and `kv_rows` the physical rows; kv_offset is then not used."""
         off = torch.as_tensor(np.asarray(b.kv_offset, np.int64), device=device)
         ln = torch.as_tensor(np.asarray(b.kv_len, np.int32), device=device)
         qs = torch.as_tensor(np.asarray(b.q_seq, np.int32), device=device)
@@ -119,9 +124,16 @@ class DeviceBatch:
         if max_q_per_seq is None:
             qsn = np.asarray(b.q_seq)
             max_q_per_seq = int(np.bincount(qsn).max()) if qsn.size else 0
+        pt = None
+        pps = 0
+        if page_size:
+            pt_host = np.ascontiguousarray(np.asarray(page_table, np.int32))
+            pps = int(pt_host.shape[1])
+            pt = torch.as_tensor(pt_host, device=device)
         st = DsaBatch(len(kv_len), len(np.asarray(b.q_pos)), max_kv_len, max_q_per_seq, kv_rows,
-                      off.data_ptr(), ln.data_ptr(), qs.data_ptr(), qp.data_ptr())
-        return cls(off, ln, qs, qp, st)
+                      off.data_ptr(), ln.data_ptr(), qs.data_ptr(), qp.data_ptr(), int(page_size), pps,
+                      pt.data_ptr() if pt is not None else None)
+        return cls(off, ln, qs, qp, st, pt)
 
 
 def workspace_size(op: int, batch: DeviceBatch, H_I: int = 64, H: int = 128, k: int = 2048, ld: int = 0) -> int:

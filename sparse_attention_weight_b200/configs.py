@@ -50,4 +50,9 @@ WORKLOADS: dict[str, Workload] = {
     "decode_128k_mtp2": Workload("decode_128k_mtp2", 5, "decode", k=2048, h_index=64,
                                  heads=128, batch=16, ctx_min=131072, ctx_max=131072,
                                  q_per_seq=2),
+    # batch-1 long-context decode (one sequence at 131072, one new token), run
+    # with a paged cache: the second decode workload of the paged-serving setting
+    "decode_b1_128k": Workload("decode_b1_128k", 6, "decode", k=2048, h_index=64,
+                               heads=128, batch=1, ctx_min=131072, ctx_max=131072,
+                               q_per_seq=1),
 }

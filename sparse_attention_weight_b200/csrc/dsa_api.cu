@@ -61,8 +61,19 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 bool batch_ok(const dsa_batch* b) {
   if (!b) return false;
   if (b->num_seqs < 1 || b->num_q < 0 || b->max_kv_len < 1 || b->max_q_per_seq < 0 || b->kv_rows < 0) return false;
-  if (b->num_q > 0 && (!b->kv_offset || !b->kv_len || !b->q_seq || !b->q_pos)) return false;
+  if (b->page_size < 0 || b->pages_per_seq < 0) return false;
+  if (b->num_q > 0) {
+    if (!b->kv_len || !b->q_seq || !b->q_pos) return false;
+    if (b->page_size == 0 ? !b->kv_offset : !b->page_table) return false;
+  }
+  if (b->page_size > 0 && static_cast<int64_t>(b->pages_per_seq) * b->page_size < b->max_kv_len) return false;
   return true;
+}
+
+// Paged caches: pages of a multiple of 64 rows (the indexer loads 64-key halves
+// of its 128-key tiles, each from one page), whole pages of physical rows.
+bool paging_ok(const dsa_batch* b) {
+  return b->page_size == 0 || (b->page_size % 64 == 0 && b->kv_rows % b->page_size == 0);
 }
 
 bool hi_ok(int H_I) { return H_I >= 4 && H_I <= 64 && H_I % 4 == 0; }
@@ -157,7 +168,7 @@ dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* 
                    static_cast<uint32_t>(hp == H_I ? G * H_I : H_I)))
     return DSA_ERR_CUDA;
   if (!make_map_2d(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, k_idx, DSA_D_INDEX,
-                   static_cast<uint64_t>(b->kv_rows > 0 ? b->kv_rows : 1), DSA_D_INDEX, 128))
+                   static_cast<uint64_t>(b->kv_rows > 0 ? b->kv_rows : 1), DSA_D_INDEX, 64))
     return DSA_ERR_CUDA;
   const int T = b->num_q;
   IndexerParams p{};
@@ -168,6 +179,10 @@ dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* 
   p.q_pos = b->q_pos;
   p.kv_offset = b->kv_offset;
   p.kv_len = b->kv_len;
+  p.page_table = b->page_table;
+  p.page_size = b->page_size;
+  p.pages_per_seq = b->pages_per_seq;
+  p.kv_rows = b->kv_rows;
   int32_t* plan = L.plan;
   p.group_q0 = plan;
   p.group_cnt = plan + T;
@@ -221,6 +236,9 @@ dsa_status run_mla(const dsa_batch* b, const uint16_t* q, const uint16_t* kv, co
   p.q_pos = b->q_pos;
   p.kv_offset = b->kv_offset;
   p.kv_len = b->kv_len;
+  p.page_table = b->page_table;
+  p.page_size = b->page_size;
+  p.pages_per_seq = b->pages_per_seq;
   p.num_seqs = b->num_seqs;
   p.kv_rows = b->kv_rows;
   p.T = b->num_q;
@@ -252,7 +270,7 @@ dsa_status dsa_indexer_scores(const dsa_batch* batch, const uint8_t* q_idx, cons
                               int H_I, float* scores, int64_t ld, void* ws, size_t ws_bytes, void* stream) {
   if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
   if (batch->num_q > 0 && (!q_idx || !k_idx || !w || !scores)) return DSA_ERR_INVALID_ARGUMENT;
-  if (!hi_ok(H_I)) return DSA_ERR_UNSUPPORTED;
+  if (!hi_ok(H_I) || !paging_ok(batch)) return DSA_ERR_UNSUPPORTED;
   if (ld < batch->max_kv_len || ld % 4 != 0) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(scores) || !aligned16(ws))
     return DSA_ERR_UNSUPPORTED;
@@ -282,7 +300,7 @@ dsa_status dsa_sparse_mla(const dsa_batch* batch, const uint16_t* q, const uint1
                           void* stream) {
   if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
   if (batch->num_q > 0 && (!q || !kv || !idx || !out)) return DSA_ERR_INVALID_ARGUMENT;
-  if (!h_ok(H) || !k_ok(k)) return DSA_ERR_UNSUPPORTED;
+  if (!h_ok(H) || !k_ok(k) || !paging_ok(batch)) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || !aligned16(ws)) return DSA_ERR_UNSUPPORTED;
   const WsLayout L = layout(ws, DSA_OP_SPARSE_MLA, batch, H, k, 0);
   if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
@@ -296,7 +314,7 @@ dsa_status dsa_forward(const dsa_batch* batch, const uint8_t* q_idx, const uint8
                        void* ws, size_t ws_bytes, void* stream) {
   if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
   if (batch->num_q > 0 && (!q_idx || !k_idx || !w || !q || !kv || !out)) return DSA_ERR_INVALID_ARGUMENT;
-  if (!hi_ok(H_I) || !h_ok(H) || !k_ok(k)) return DSA_ERR_UNSUPPORTED;
+  if (!hi_ok(H_I) || !h_ok(H) || !k_ok(k) || !paging_ok(batch)) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(q) || !aligned16(kv) ||
       !aligned16(out) || !aligned16(ws))
     return DSA_ERR_UNSUPPORTED;
@@ -387,7 +405,7 @@ extern "C" dsa_status dsa_indexer_scores_noalloc(const dsa_batch* batch, const u
                                                  int64_t ld, void* stream) {
   if (!batch_ok(batch)) return DSA_ERR_INVALID_ARGUMENT;
   if (batch->num_q > 0 && (!q_idx || !k_idx || !w || !scores)) return DSA_ERR_INVALID_ARGUMENT;
-  if (!hi_ok(H_I)) return DSA_ERR_UNSUPPORTED;
+  if (!hi_ok(H_I) || !paging_ok(batch)) return DSA_ERR_UNSUPPORTED;
   if (batch->num_q > DSA_NOALLOC_MAX_Q) return DSA_ERR_UNSUPPORTED;
   if (ld < batch->max_kv_len || ld % 4 != 0) return DSA_ERR_UNSUPPORTED;
   if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(scores)) return DSA_ERR_UNSUPPORTED;

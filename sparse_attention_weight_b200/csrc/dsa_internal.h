@@ -14,8 +14,12 @@ struct IndexerParams {
   int64_t ld;
   const int32_t* q_seq;      // [T]
   const int32_t* q_pos;      // [T]
-  const int64_t* kv_offset;  // [B]
+  const int64_t* kv_offset;  // [B] (contiguous layout)
   const int32_t* kv_len;     // [B]
+  const int32_t* page_table; // [B, pages_per_seq] (paged layout, page_size > 0)
+  int page_size;             // 0 = contiguous rows from kv_offset
+  int pages_per_seq;
+  int64_t kv_rows;           // rows of the k_idx buffer
   // plan (workspace)
   int32_t* group_q0;         // [T]
   int32_t* group_cnt;        // [T]
@@ -56,8 +60,11 @@ struct MlaParams {
   float* lse;                // [T, H] or null
   const int32_t* q_seq;
   const int32_t* q_pos;
-  const int64_t* kv_offset;
+  const int64_t* kv_offset;  // contiguous layout
   const int32_t* kv_len;
+  const int32_t* page_table; // [B, pages_per_seq] (paged layout, page_size > 0)
+  int page_size;             // 0 = contiguous rows from kv_offset
+  int pages_per_seq;
   int num_seqs;
   int64_t kv_rows;
   int T;

@@ -107,14 +107,17 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         int g = find_group(p.item_off, ngroups, i0);
         int g_lo = p.item_off[g], g_hi = p.item_off[g + 1];
         int prev_g = -1, issued = 0, gq = 0;   // gq: query tiles loaded (buffer gq & 1)
-        int64_t row_base = 0;                   // first cache row of the group's sequence
+        int64_t row_base = 0;                   // first cache row of the group's sequence (contiguous)
+        int seq_g = 0, len_g = 0;               // the group's sequence and its length
         int st = 0;                             // key-ring stage and its phase, advanced per item
         uint32_t ph = 0;
         for (int i = i0; i < i1; ++i) {
           while (g_hi <= i) { ++g; g_lo = g_hi; g_hi = p.item_off[g + 1]; }
           const int kt = i - g_lo;
           if (g != prev_g) {
-            row_base = p.kv_offset[p.group_seq[g]];
+            seq_g = p.group_seq[g];
+            len_g = p.kv_len[seq_g];
+            row_base = p.page_size == 0 ? p.kv_offset[seq_g] : 0;
             // two query buffers: the tile of group gq reuses the buffer of group
             // gq - 2, whose MMAs must have completed; the previous group's MMAs may
             // still be running meanwhile
@@ -132,8 +135,27 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           }
           if (!mbar_wait(&S.k_empty[st], ph ^ 1, p.status, abort_flag)) break;
           mbar_arrive_expect_tx(&S.k_full[st], kTileBytes);
-          const int64_t row = row_base + static_cast<int64_t>(kt) * kKeyTile;
-          tma_load_2d(S.k[st], &tm_k, &S.k_full[st], 0, static_cast<int>(row));
+          // the tile's two halves of 64 keys; with a paged cache each half lies in
+          // one page (pages hold a multiple of 64 rows)
+          int64_t row0 = 0;
+          for (int h = 0; h < 2; ++h) {
+            const int key0 = kt * kKeyTile + h * 64;
+            int64_t row = row_base + key0;
+            if (p.page_size != 0) {
+              if (key0 < len_g) {
+                const int pg = p.page_table[static_cast<int64_t>(seq_g) * p.pages_per_seq + key0 / p.page_size];
+                row = static_cast<int64_t>(pg) * p.page_size + key0 % p.page_size;
+                if (pg < 0 || static_cast<int64_t>(pg + 1) * p.page_size > p.kv_rows) {
+                  set_status(p.status, DSA_DEV_BAD_INDEX);
+                  row = 0;
+                }
+              } else {
+                row = row0;                     // keys past the sequence end are masked
+              }
+            }
+            if (h == 0) row0 = row;
+            tma_load_2d(S.k[st] + h * 64 * DSA_D_INDEX, &tm_k, &S.k_full[st], 0, static_cast<int>(row));
+          }
           ++issued;
           if (++st == kStages) { st = 0; ph ^= 1; }
         }
@@ -340,9 +362,14 @@ __device__ __forceinline__ int visible_keys(const IndexerParams& p, int t, int B
   const int seq = p.q_seq[t];
   if (seq < 0 || seq >= B) return -1;
   const int len = p.kv_len[seq];
-  const int64_t off = p.kv_offset[seq];
   const int pos = p.q_pos[t];
-  if (len < 0 || len > p.max_kv_len || off < 0 || off + len > kv_rows || pos < 0 || pos >= len) return -1;
+  if (len < 0 || len > p.max_kv_len || pos < 0 || pos >= len) return -1;
+  if (p.page_size == 0) {
+    const int64_t off = p.kv_offset[seq];
+    if (off < 0 || off + len > kv_rows) return -1;
+  } else if (len > static_cast<int64_t>(p.pages_per_seq) * p.page_size) {
+    return -1;
+  }
   return pos + 1;
 }
 

@@ -187,7 +187,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
   const int head0 = static_cast<int>(rank) * kHeads;       // first head of this CTA
 
   struct Item {
-    int t, split, len;
+    int t, split, seq, len;
     int64_t base;
     bool ok;
     const int32_t* idx_row;
@@ -199,11 +199,26 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
     I.split = it % p.splits;
     const int seq = p.q_seq[I.t];
     const bool seq_ok = seq >= 0 && seq < p.num_seqs;
+    I.seq = seq_ok ? seq : 0;
     I.len = seq_ok ? p.kv_len[seq] : 0;
-    I.base = seq_ok ? p.kv_offset[seq] : 0;
-    I.ok = seq_ok && I.len >= 0 && I.base >= 0 && I.base + I.len <= p.kv_rows;
+    I.base = seq_ok && p.page_size == 0 ? p.kv_offset[seq] : 0;
+    I.ok = seq_ok && I.len >= 0 &&
+           (p.page_size == 0 ? I.base >= 0 && I.base + I.len <= p.kv_rows
+                             : I.len <= static_cast<int64_t>(p.pages_per_seq) * p.page_size);
     I.idx_row = p.idx + static_cast<int64_t>(I.t) * p.k;
     return I;
+  };
+  // cache row of the usable local index v (0 <= v < len), -1 (flagged) when its
+  // page points outside the cache
+  auto cache_row = [&](const Item& I, int v) -> int64_t {
+    if (p.page_size == 0) return I.base + v;
+    const int pg = __ldg(p.page_table + static_cast<int64_t>(I.seq) * p.pages_per_seq + v / p.page_size);
+    const int64_t r = static_cast<int64_t>(pg) * p.page_size + v % p.page_size;
+    if (pg < 0 || r >= p.kv_rows) {
+      set_status(p.status, DSA_DEV_BAD_INDEX);
+      return -1;
+    }
+    return r;
   };
   // blocks of 256 entries covering the used part of the index row, split evenly
   auto plan_of = [&](int b, int split, int& blk0, int& nblk) {
@@ -517,16 +532,16 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       plan_of(b, I.split, blk0, nblk);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.plan_free[b]);
-      // rows of this lane's rows (16gw + 4i + rsub) of block bk, -1 if unusable
-      auto rows_of = [&](int bk, int (&rr)[4]) {
+      // cache rows of this lane's rows (16gw + 4i + rsub) of block bk, -1 if unusable
+      auto rows_of = [&](int bk, int64_t (&rr)[4]) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int e = bk * kBlk + static_cast<int>(rank) * kRows + 16 * gw + 4 * i + rsub;
           const int v = e < p.k ? __ldg(I.idx_row + e) : -1;
-          rr[i] = (v >= 0 && v < I.len) ? v : -1;
+          rr[i] = (v >= 0 && v < I.len) ? cache_row(I, v) : -1;
         }
       };
-      int cur[4], nxt[4];
+      int64_t cur[4], nxt[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) { cur[i] = -1; nxt[i] = -1; }
       if (nblk > 0) rows_of(blk0, cur);
@@ -534,7 +549,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         if (j + 1 < nblk) rows_of(blk0 + j + 1, nxt);
         const uint16_t* src[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) src[h] = p.kv + (cur[h] < 0 ? 0 : I.base + cur[h]) * DSA_D_QK + c16 * 8;
+        for (int h = 0; h < 4; ++h) src[h] = p.kv + (cur[h] < 0 ? 0 : cur[h]) * DSA_D_QK + c16 * 8;
         for (int i = 0; i < kDChunks; ++i) {
           const int c = chunk_at(i);
           if (!warp_wait(&S.s_empty[slot], sph ^ 1, p.status, ab, false)) { ok = false; break; }
@@ -578,12 +593,12 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       plan_of(b, I.split, blk0, nblk);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.plan_free[b]);
-      auto row_of = [&](int bk) -> int {
+      auto row_of = [&](int bk) -> int64_t {
         const int e = bk * kBlk + (lane >> 2) * kVRows + 4 * vw + (lane & 3);
         const int v = e < p.k ? __ldg(I.idx_row + e) : -1;
-        return (v >= 0 && v < I.len) ? v : -1;
+        return (v >= 0 && v < I.len) ? cache_row(I, v) : -1;
       };
-      int cur = nblk > 0 ? row_of(blk0) : -1, nxt = -1;
+      int64_t cur = nblk > 0 ? row_of(blk0) : -1, nxt = -1;
       for (int j = 0; j < nblk && ok; ++j) {
         if (j + 1 < nblk) nxt = row_of(blk0 + j + 1);
         for (int vs = 0; vs < kVSlices; ++vs) {
@@ -591,10 +606,10 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
           const uint32_t dst0 = smem_u32(S.v_ring[slot][g]);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const int v = __shfl_sync(0xffffffffu, cur, vs * 4 + i);
+            const int64_t v = __shfl_sync(0xffffffffu, cur, vs * 4 + i);
             const int r = 4 * vw + i;                          // row of the slice
             cp_async16(dst0 + r * 128 + ((c16 ^ (r & 7)) << 4),
-                       p.kv + (v < 0 ? 0 : I.base + v) * DSA_D_QK + dim0, v < 0 ? 0u : 16u);
+                       p.kv + (v < 0 ? 0 : v) * DSA_D_QK + dim0, v < 0 ? 0u : 16u);
           }
           cp_async_arrive_noinc(&S.v_loaded[slot]);
           if (++slot == kVStages) { slot = 0; vph ^= 1; }

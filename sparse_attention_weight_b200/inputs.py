@@ -198,6 +198,31 @@ def cache_rows(wl: Workload, batch: Batch, which: str, seed: int = 0,
     return np.concatenate(parts, axis=0) if parts else np.empty((0,) + shape, np.uint8)
 
 
+def paged_layout(batch: Batch, page_size: int, seed: int = 0, spare_pages: int = 3):
+    """A paged storage layout of the batch's caches (the block-table layout of
+    paged inference caches): every sequence's rows cut into pages of
+    `page_size`, the pages scattered over a physical pool in a seeded random
+    order with a few unused pages.  Returns (page_table int32 [B, pages_per_seq],
+    unused entries -1; src int64 [pool rows]: the contiguous row each physical
+    row holds, -1 for padding).  Storage only: no values are computed."""
+    lens = batch.kv_len.astype(np.int64)
+    npages = (lens + page_size - 1) // page_size
+    pps = int(max(1, (batch.max_kv_len + page_size - 1) // page_size))
+    total = int(npages.sum()) + spare_pages
+    perm = np.random.default_rng([seed, 7001, page_size]).permutation(total)
+    table = np.full((batch.num_seqs, pps), -1, np.int32)
+    src = np.full(total * page_size, -1, np.int64)
+    k = 0
+    for b in range(batch.num_seqs):
+        for i in range(int(npages[b])):
+            phys = int(perm[k])
+            k += 1
+            table[b, i] = phys
+            n = int(min(page_size, lens[b] - i * page_size))
+            src[phys * page_size: phys * page_size + n] = batch.kv_offset[b] + i * page_size + np.arange(n)
+    return table, src
+
+
 def make_inputs(wl: Workload, seed: int = 0, chunk_index: int | None = None) -> dict:
     """Every input of one call of the workload, as host numpy arrays."""
     batch = make_batch(wl, seed, chunk_index)

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_function(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.dsa_abi_version() == 1
+    assert lib.dsa_abi_version() == 2
     for code, name in B.STATUS_NAMES.items():
         assert lib.dsa_status_string(code).decode() == name
 
@@ -82,6 +82,33 @@ def test_host_argument_checks(lib):
     assert lib.dsa_topk(ctypes.byref(bad), p, 3000, 2048, p, ws, big, None) == 1
     nulls = B.DsaBatch(2, 16, 3000, 0, 6000, 0, 0, 0, 0)
     assert lib.dsa_topk(ctypes.byref(nulls), p, 3000, 2048, p, ws, big, None) == 1
+
+
+def test_paged_layout_host_checks(lib):
+    """Paged caches (the block-table layout of paged inference caches): the page
+    size must be a multiple of 64 dividing the physical rows, the page table
+    must be given and cover max_kv_len; kv_offset is then not needed."""
+    ws, p, big = 0x50000, 0x60000, 1 << 40
+    pt = 0x70000
+
+    def paged(page_size, pps, table=pt, kv_rows=8192, max_len=3000):
+        return B.DsaBatch(2, 16, max_len, 0, kv_rows, 0, 0x20000, 0x30000, 0x40000, page_size, pps, table)
+
+    sz = lambda b: lib.dsa_workspace_size(B.OP_FORWARD, ctypes.byref(b), 64, 128, 2048, 0)
+    assert sz(paged(64, 47)) > 0                      # 47 * 64 = 3008 >= 3000
+    assert sz(paged(64, 46)) == 0                     # 2944 < max_kv_len
+    assert sz(paged(64, 47, table=0)) == 0            # no page table
+    assert sz(B.DsaBatch(2, 16, 3000, 0, 8192, 0, 0x20000, 0x30000, 0x40000, -64, 47, pt)) == 0
+    # unsupported page sizes: not a multiple of 64, or not dividing the physical rows
+    for ps, pps in ((32, 94), (96, 32)):
+        b = paged(ps, pps)
+        assert lib.dsa_indexer_scores(ctypes.byref(b), p, p, p, 64, p, 3000, ws, big, None) == 2
+        assert lib.dsa_sparse_mla(ctypes.byref(b), p, p, p, 2048, 128, 0.1, p, None, ws, big, None) == 2
+        assert lib.dsa_forward(ctypes.byref(b), p, p, p, 64, p, p, 128, 2048, 0.1, p, None, ws, big, None) == 2
+    b = paged(128, 24, kv_rows=8000)                  # 8000 rows is not whole pages of 128
+    assert lib.dsa_sparse_mla(ctypes.byref(b), p, p, p, 2048, 128, 0.1, p, None, ws, big, None) == 2
+    # the top-k reads no cache rows: any valid paged batch is accepted on the host
+    assert lib.dsa_topk(ctypes.byref(paged(32, 94)), p, 3000, 2048, p, ws, 0, None) == 3
 
 
 def test_read_device_status_rejects_null(lib):
