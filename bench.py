@@ -406,6 +406,62 @@ def sub_record(wl, args, rank, world, device, peaks) -> dict:
     return rec
 
 
+def project_record(args, device, peaks, seed: int) -> dict:
+    """The step before the path (dsa_project_append) on the last 4096-token chunk
+    of the 64K prefill: d_model 7168, H_I 64, H 128, appended to a 65536-row cache.
+    One call = the stacked projection GEMM (cuBLASLt) + the RoPE/cast/append kernel."""
+    import torch
+
+    from sparse_attention_weight_b200 import binding as B
+    from sparse_attention_weight_b200 import inputs
+    T, d, H_I, H, rows = 4096, 7168, 64, 128, 65536
+    n_all = H_I * D_INDEX + D_INDEX + H_I + D_QK + H * D_QK
+    pos = np.arange(rows - T, rows, dtype=np.int32)
+    bh = inputs.Batch(np.zeros(1, np.int64), np.array([rows], np.int32), np.zeros(T, np.int32), pos,
+                      np.arange(T, dtype=np.int32))
+    db = B.DeviceBatch.from_host(bh, device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 7919 + 7100)
+    hidden = torch.randn((T, d), generator=g, device=device).to(torch.bfloat16).view(torch.int16)
+    w_all = (torch.randn((n_all, d), generator=g, device=device) / np.sqrt(d)).to(torch.bfloat16).view(torch.int16)
+    q_idx = torch.empty((T, H_I, D_INDEX), dtype=torch.uint8, device=device)
+    w = torch.empty((T, H_I), dtype=torch.float32, device=device)
+    q = torch.empty((T, H, D_QK), dtype=torch.int16, device=device)
+    k_cache = torch.zeros((rows, D_INDEX), dtype=torch.uint8, device=device)
+    kv_cache = torch.zeros((rows, D_QK), dtype=torch.int16, device=device)
+    ws = B.workspace(B.OP_PROJECT, db, H_I=H_I, H=H, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    run = lambda: B.dsa_project_append(db, hidden, w_all, d, H_I, H, 10000.0, q_idx, w, q, k_cache, kv_cache, ws)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize()
+    if B.read_device_status(ws):
+        raise RuntimeError("device status flags in dsa_project_append")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    l0 = B.launch_count()
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record()
+        run()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+    flop = 2.0 * T * d * n_all
+    # the epilogue kernel's algorithmic bytes: fp32 projections in, stored outputs and cache rows out
+    epi_bytes = T * n_all * 4 + T * (H_I * D_INDEX + H_I * 4 + H * D_QK * 2) + T * (D_INDEX + D_QK * 2)
+    return {"metric": "projection + RoPE + cache append tokens/s", "value": T / (ms / 1e3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": args.steps, "calls_per_step": 1, "queries_per_step": T,
+            "config": {"workload": "project_append_4k", "tokens": T, "d_model": d, "h_index": H_I, "heads": H,
+                       "cache_rows": rows, "l2": "flushed before every timed step (512 MB write)"},
+            "stages": {"gemm_plus_epilogue": {"ms": ms, "tflops": flop / (ms / 1e3) / 1e12,
+                                              "bf16_frac": flop / (ms / 1e3) / 1e12 / peaks["bf16"]},
+                       "epilogue_algorithmic_bytes": epi_bytes},
+            "gpu_launches": B.launch_count() - l0,
+            "data": "synthetic, drawn on the device (seeded Philox); GEMM by cuBLASLt (a plain library GEMM), "
+                    "RoPE / casts / append by the library's own kernel"}
+
+
 def config_of(wl, args) -> dict:
     decode = wl.kind == "decode"
     return {"workload": wl.name, "k": wl.k, "h_index": wl.h_index, "heads": wl.heads, "d_qk": D_QK, "d_v": D_V,
@@ -618,6 +674,8 @@ def main():
         for name in ("decode_b64", "decode_128k_mtp2", "decode_b1_128k", "chunked_64k"):
             if name != wl.name:
                 line["workloads"][name] = sub_record(WORKLOADS[name], args, rank, world, device, peaks)
+        line["workloads"]["project_append_4k"] = project_record(args, device, peaks, rank_seed(rank))
+        torch.cuda.empty_cache()
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline(wl)

@@ -96,6 +96,7 @@ typedef struct dsa_batch {
 #define DSA_OP_TOPK 1
 #define DSA_OP_SPARSE_MLA 2
 #define DSA_OP_FORWARD 3
+#define DSA_OP_PROJECT 4
 
 /*
  * Bytes of workspace `ws` an operation needs (always >= 256: the status word and
@@ -104,6 +105,41 @@ typedef struct dsa_batch {
  * Returns 0 for an invalid op or batch.
  */
 size_t dsa_workspace_size(int op, const dsa_batch *batch, int H_I, int H, int k, int64_t ld);
+
+/*
+ * The step before the path ("四步工作流程" 第一步 查詢與鍵的投影: queries, keys and
+ * per-head weights projected from the hidden states with rotary embeddings;
+ * "DeepSeek 稀疏注意力路线", V3's MLA: the latent down-projection that is cached and
+ * the decoupled RoPE channel): projections of the T new tokens, RoPE, storage casts
+ * and cache append, with the caller's (e.g. synthetic) weights.
+ *   hidden (device) bf16 bits [T, d_model]
+ *   w_all  (device) bf16 bits [N, d_model], N = H_I*128 + 128 + H_I + 512 + 64 + H*576,
+ *          stacked rows for: the indexer query heads (H_I x 128), the indexer key
+ *          (128), the per-head weights (H_I), the latent (512), the RoPE key (64),
+ *          the latent query heads (H x 512), the RoPE query heads (H x 64)
+ *   Y = hidden W^T in fp32 (tensor cores, fp32 accumulation), then for token t at
+ *   position pos = q_pos[t] of sequence b = q_seq[t]:
+ *   q_idx (device) E4M3 [T, H_I, 128]: RoPE of each indexer query head
+ *   w     (device) fp32 [T, H_I]: the per-head weights
+ *   q     (device) bf16 bits [T, H, 576]: per head [latent query, RoPE of the RoPE query]
+ *   k_idx (device) E4M3 [kv_rows, 128]: the cache row of key pos of sequence b (see
+ *         dsa_batch) receives the RoPE of the indexer key
+ *   kv    (device) bf16 bits [kv_rows, 576]: the same row receives [latent, RoPE of
+ *         the RoPE key]; no other cache row is written
+ * RoPE rotates the pairs (x[2i], x[2i+1]) of a D-dim part (D = 128 for the indexer,
+ * 64 for the MLA) by the angle pos * rope_base^(-2i/D), computed in double
+ * precision.  E4M3 rounds to nearest even and saturates at +-448; bf16 rounds to
+ * nearest even.  A token outside its sequence (q_seq/q_pos out of range) flags
+ * DSA_DEV_BAD_QUERY, one whose cache row lies outside kv_rows DSA_DEV_BAD_INDEX;
+ * such tokens are not appended.
+ * Workspace: dsa_workspace_size(DSA_OP_PROJECT, batch, H_I, H, 0, 0) (the fp32
+ * projections and the GEMM's scratch).
+ * Supported: H_I in {4, 8, ..., 64}, H in {8, 16, ..., 128}, d_model a multiple of
+ * 8, every buffer 16-byte aligned.  DSA_ERR_CUDA if the GEMM library fails.
+ */
+dsa_status dsa_project_append(const dsa_batch *batch, const uint16_t *hidden, const uint16_t *w_all, int d_model,
+                              int H_I, int H, float rope_base, uint8_t *q_idx, float *w, uint16_t *q,
+                              uint8_t *k_idx, uint16_t *kv, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Step 1, lightning indexer ("四步工作流程" 第二步 索引器評分; "两阶段流程" 1).

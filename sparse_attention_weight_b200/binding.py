@@ -21,11 +21,11 @@ DSA_OK = 0
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARGUMENT", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_WORKSPACE_TOO_SMALL", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_DEVICE"}
 DEV_BAD_QUERY, DEV_BAD_INDEX, DEV_TIMEOUT = 1, 2, 4
-OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD = 0, 1, 2, 3
+OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_PROJECT = 0, 1, 2, 3, 4
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward",
            "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
-           "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout", "dsa_launch_count")
+           "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout", "dsa_launch_count", "dsa_project_append")
 NOALLOC_MAX_Q = 16384
 
 
@@ -66,6 +66,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_mla.argtypes = [bp, vp, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
         L.dsa_forward.argtypes = [bp, vp, vp, vp, i32, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
         L.dsa_indexer_scores_noalloc.argtypes = [bp, vp, vp, vp, i32, vp, i64, vp]
+        L.dsa_project_append.argtypes = [bp, vp, vp, i32, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
         L.dsa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
         L.dsa_forward_ws_views.argtypes = [bp, i32, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(i64),
                                            ctypes.POINTER(vp)]
@@ -75,7 +76,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_abi_version.restype = i32
         L.dsa_launch_count.restype = ctypes.c_uint64
         for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward", "dsa_forward_ws_views",
-                   "dsa_read_device_status", "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout"):
+                   "dsa_read_device_status", "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout",
+                   "dsa_project_append"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -174,6 +176,13 @@ def dsa_sparse_mla(batch: DeviceBatch, q, kv, idx, k: int, H: int, sm_scale: flo
     _check("dsa_sparse_mla", lib().dsa_sparse_mla(
         ctypes.byref(batch.struct), _ptr(q), _ptr(kv), _ptr(idx), k, H, sm_scale, _ptr(out), _ptr(lse), _ptr(ws),
         ws.numel(), _stream(stream)))
+
+
+def dsa_project_append(batch: DeviceBatch, hidden, w_all, d_model: int, H_I: int, H: int, rope_base: float, q_idx,
+                       w, q, k_idx, kv, ws, stream=None):
+    _check("dsa_project_append", lib().dsa_project_append(
+        ctypes.byref(batch.struct), _ptr(hidden), _ptr(w_all), d_model, H_I, H, rope_base, _ptr(q_idx), _ptr(w),
+        _ptr(q), _ptr(k_idx), _ptr(kv), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def dsa_forward(batch: DeviceBatch, q_idx, k_idx, w, H_I: int, q, kv, H: int, k: int, sm_scale: float, out, lse,

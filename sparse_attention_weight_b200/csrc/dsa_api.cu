@@ -113,6 +113,8 @@ int mla_splits(const dsa_batch* b, int k) {
   return s;
 }
 
+int proj_rows(int H_I, int H) { return H_I * DSA_D_INDEX + DSA_D_INDEX + H_I + DSA_D_QK + H * DSA_D_QK; }
+
 size_t plan_bytes(const dsa_batch* b) { return align_up((6 * static_cast<size_t>(b->num_q) + 2) * sizeof(int32_t)); }
 
 struct WsLayout {
@@ -124,6 +126,26 @@ struct WsLayout {
   int32_t* idx;
   size_t bytes;
 };
+
+struct ProjLayout {
+  uint32_t* status;
+  float* y;
+  void* gemm_ws;
+  size_t bytes;
+};
+
+ProjLayout proj_layout(void* ws, const dsa_batch* b, int H_I, int H) {
+  ProjLayout L{};
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  size_t off = kWsHeader;
+  L.status = reinterpret_cast<uint32_t*>(p);
+  L.y = reinterpret_cast<float*>(p + off);
+  off += align_up(static_cast<size_t>(b->num_q) * proj_rows(H_I, H) * sizeof(float));
+  L.gemm_ws = p + off;
+  off += project_gemm_workspace_bytes();
+  L.bytes = off;
+  return L;
+}
 
 WsLayout layout(void* ws, int op, const dsa_batch* b, int H, int k, int64_t ld) {
   WsLayout L{};
@@ -257,8 +279,8 @@ using namespace dsa;
 extern "C" {
 
 size_t dsa_workspace_size(int op, const dsa_batch* batch, int H_I, int H, int k, int64_t ld) {
-  (void)H_I;
   if (!batch_ok(batch)) return 0;
+  if (op == DSA_OP_PROJECT) return hi_ok(H_I) && h_ok(H) ? proj_layout(nullptr, batch, H_I, H).bytes : 0;
   if (op < DSA_OP_INDEXER || op > DSA_OP_FORWARD) return 0;
   if ((op == DSA_OP_SPARSE_MLA || op == DSA_OP_FORWARD) && (!h_ok(H) || !k_ok(k))) return 0;
   if (op == DSA_OP_FORWARD && !k_ok(k)) return 0;
@@ -328,6 +350,50 @@ dsa_status dsa_forward(const dsa_batch* batch, const uint8_t* q_idx, const uint8
   s = run_topk(batch, L.scores, ld, k, L.idx, L, st);
   if (s != DSA_OK) return s;
   return run_mla(batch, q, kv, L.idx, k, H, sm_scale, out, lse, L, st);
+}
+
+dsa_status dsa_project_append(const dsa_batch* batch, const uint16_t* hidden, const uint16_t* w_all, int d_model,
+                              int H_I, int H, float rope_base, uint8_t* q_idx, float* w, uint16_t* q,
+                              uint8_t* k_idx, uint16_t* kv, void* ws, size_t ws_bytes, void* stream) {
+  if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!hidden || !w_all || !q_idx || !w || !q || !k_idx || !kv))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (d_model <= 0 || !(rope_base > 0.f)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!hi_ok(H_I) || !h_ok(H) || d_model % 8 != 0 || !paging_ok(batch)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(hidden) || !aligned16(w_all) || !aligned16(q_idx) || !aligned16(w) || !aligned16(q) ||
+      !aligned16(k_idx) || !aligned16(kv) || !aligned16(ws))
+    return DSA_ERR_UNSUPPORTED;
+  const ProjLayout L = proj_layout(ws, batch, H_I, H);
+  if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (batch->num_q == 0) return DSA_OK;
+  ProjParams p{};
+  p.y = L.y;
+  p.q_idx = q_idx;
+  p.w = w;
+  p.q = q;
+  p.k_cache = k_idx;
+  p.kv_cache = kv;
+  p.q_seq = batch->q_seq;
+  p.q_pos = batch->q_pos;
+  p.kv_offset = batch->kv_offset;
+  p.kv_len = batch->kv_len;
+  p.page_table = batch->page_table;
+  p.page_size = batch->page_size;
+  p.pages_per_seq = batch->pages_per_seq;
+  p.num_seqs = batch->num_seqs;
+  p.kv_rows = batch->kv_rows;
+  p.T = batch->num_q;
+  p.n_all = proj_rows(H_I, H);
+  p.hi = H_I;
+  p.heads = H;
+  p.rope_base = rope_base;
+  p.status = L.status;
+  bool gemm_failed = false;
+  const cudaError_t e = launch_project(p, hidden, w_all, d_model, L.gemm_ws, project_gemm_workspace_bytes(), st,
+                                       &gemm_failed);
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status dsa_forward_ws_views(const dsa_batch* batch, int H_I, int H, int k, void* ws, float** scores, int64_t* ld,

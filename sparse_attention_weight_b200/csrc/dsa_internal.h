@@ -74,9 +74,36 @@ struct MlaParams {
   uint32_t* status;
 };
 
+struct ProjParams {
+  float* y;                  // [T, n_all] fp32 projections (workspace)
+  uint8_t* q_idx;            // [T, H_I, 128] E4M3
+  float* w;                  // [T, H_I]
+  uint16_t* q;               // [T, H, 576] bf16
+  uint8_t* k_cache;          // [kv_rows, 128] E4M3
+  uint16_t* kv_cache;        // [kv_rows, 576] bf16
+  const int32_t* q_seq;
+  const int32_t* q_pos;
+  const int64_t* kv_offset;  // contiguous layout
+  const int32_t* kv_len;
+  const int32_t* page_table; // paged layout (page_size > 0)
+  int page_size;
+  int pages_per_seq;
+  int num_seqs;
+  int64_t kv_rows;
+  int T;
+  int n_all;                 // rows of the stacked projection matrix
+  int hi;                    // H_I
+  int heads;                 // H
+  float rope_base;
+  uint32_t* status;
+};
+
 // Counts kernel launches made by the library (dsa_launch_count).
 void count_launches(int n);
 
+size_t project_gemm_workspace_bytes();
+cudaError_t launch_project(const ProjParams& p, const uint16_t* hidden, const uint16_t* w_all, int d_model,
+                           void* gemm_ws, size_t gemm_ws_bytes, cudaStream_t stream, bool* gemm_failed);
 size_t indexer_smem_bytes();
 size_t mla_smem_bytes();
 cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int hi_pad,

@@ -223,6 +223,17 @@ def paged_layout(batch: Batch, page_size: int, seed: int = 0, spare_pages: int =
     return table, src
 
 
+def projection_inputs(T: int, d_model: int, n_rows: int, seed: int = 0) -> dict:
+    """Hidden states ~ N(0,1) and a stacked projection matrix ~ N(0, 1/d_model)
+    (so every projection is ~ N(0,1), the distribution of the path's inputs), as
+    bf16 bits: hidden [T, d_model], w_all [n_rows, d_model]."""
+    rng_h = np.random.default_rng([seed, 7100, T, d_model])
+    rng_w = np.random.default_rng([seed, 7101, n_rows, d_model])
+    h = rng_h.standard_normal((T, d_model), dtype=np.float32)
+    w = rng_w.standard_normal((n_rows, d_model), dtype=np.float32) * np.float32(1.0 / np.sqrt(d_model))
+    return {"hidden": to_bf16_bits(h), "w_all": to_bf16_bits(w)}
+
+
 def make_inputs(wl: Workload, seed: int = 0, chunk_index: int | None = None) -> dict:
     """Every input of one call of the workload, as host numpy arrays."""
     batch = make_batch(wl, seed, chunk_index)

@@ -111,6 +111,23 @@ def test_paged_layout_host_checks(lib):
     assert lib.dsa_topk(ctypes.byref(paged(32, 94)), p, 3000, 2048, p, ws, 0, None) == 3
 
 
+def test_project_append_host_checks(lib):
+    b = _fake_batch()
+    ws, p, big = 0x50000, 0x60000, 1 << 40
+    sz = lib.dsa_workspace_size(B.OP_PROJECT, ctypes.byref(b), 64, 128, 0, 0)
+    n_all = 64 * 128 + 128 + 64 + 576 + 128 * 576
+    assert sz >= 256 + 16 * n_all * 4                 # the fp32 projections of the 16 tokens
+    assert lib.dsa_workspace_size(B.OP_PROJECT, ctypes.byref(b), 10, 128, 0, 0) == 0
+    call = lambda **kw: lib.dsa_project_append(ctypes.byref(b), kw.get("h", p), p, kw.get("d", 7168),
+                                               kw.get("hi", 64), kw.get("H", 128), kw.get("base", 10000.0),
+                                               p, p, p, p, p, ws, kw.get("ws_bytes", big), None)
+    assert call(h=0) == 1                             # null input
+    assert call(d=0) == 1 and call(base=0.0) == 1
+    assert call(hi=10) == 2 and call(H=12) == 2 and call(d=7170) == 2
+    assert call(h=p + 4) == 2                         # alignment
+    assert call(ws_bytes=1024) == 3
+
+
 def test_read_device_status_rejects_null(lib):
     flags = ctypes.c_uint32()
     assert lib.dsa_read_device_status(None, ctypes.byref(flags), None) == 1
