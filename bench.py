@@ -212,7 +212,7 @@ class Call:
     """Device buffers and workspaces of one call (one batch) of the path."""
 
     def __init__(self, wl, bh, dev: dict, device, out=None, lse=None, kv_rows=None, scores=None, idx=None,
-                 page_size=0, page_table=None):
+                 page_size=0, page_table=None, fused_hist=False):
         import torch
 
         from sparse_attention_weight_b200 import binding as B
@@ -229,6 +229,10 @@ class Call:
         self.out = out if out is not None else torch.empty((T, wl.heads, D_V), dtype=torch.int16, device=device)
         self.lse = lse if lse is not None else torch.empty((T, wl.heads), dtype=torch.float32, device=device)
         self.ws_i = B.workspace(B.OP_INDEXER, self.db, H_I=wl.h_index, ld=self.ld, device=device)
+        # indexer -> top-k fused through the key histogram (measured separately; the
+        # default path is unfused, which is faster here)
+        self.hist = (torch.empty((T, 2048), dtype=torch.int32, device=device)
+                     if fused_hist and B.topk_uses_hist(self.db, wl.k) else None)
         self.ws_t = B.workspace(B.OP_TOPK, self.db, k=wl.k, device=device)
         self.ws_m = B.workspace(B.OP_SPARSE_MLA, self.db, H=wl.heads, k=wl.k, device=device)
         self.idx_pairs, self.sel_pairs = algorithmic_pairs(bh.q_pos, wl.k)
@@ -239,11 +243,18 @@ class Call:
         B, wl, d = self.B, self.wl, self.dev
         if ev is not None:
             ev[base].record(stream)
-        B.dsa_indexer_scores(self.db, d["q_idx"], d["k_idx"], d["w"], wl.h_index, self.scores, self.ld, self.ws_i,
-                             stream)
+        if self.hist is not None:
+            B.dsa_indexer_scores_hist(self.db, d["q_idx"], d["k_idx"], d["w"], wl.h_index, self.scores, self.ld,
+                                      self.hist, self.ws_i, stream)
+        else:
+            B.dsa_indexer_scores(self.db, d["q_idx"], d["k_idx"], d["w"], wl.h_index, self.scores, self.ld,
+                                 self.ws_i, stream)
         if ev is not None:
             ev[base + 1].record(stream)
-        B.dsa_topk(self.db, self.scores, self.ld, wl.k, self.idx, self.ws_t, stream)
+        if self.hist is not None:
+            B.dsa_topk_hist(self.db, self.scores, self.ld, self.hist, wl.k, self.idx, self.ws_t, stream)
+        else:
+            B.dsa_topk(self.db, self.scores, self.ld, wl.k, self.idx, self.ws_t, stream)
         if ev is not None:
             ev[base + 2].record(stream)
         B.dsa_sparse_mla(self.db, d["q"], d["kv"], self.idx, wl.k, wl.heads, wl.sm_scale, self.out, self.lse,
@@ -347,7 +358,7 @@ def host_call(wl, device, seed, chunk=None):
     return Call(wl, ins["batch"], dev, device), ins
 
 
-def device_calls(wl, device, seed):
+def device_calls(wl, device, seed, fused_hist=False):
     """The calls of one step of a workload with device-drawn inputs (a chunked
     prefill: one call per chunk against the growing cache prefix)."""
     import torch
@@ -382,13 +393,13 @@ def device_calls(wl, device, seed):
             pool[used] = dev[name][src_t[used]]
             dev[name] = pool
         return [Call(wl, bh, dev, device, kv_rows=src.size, page_size=ps, page_table=table)]
-    return [Call(wl, bh, dev, device)]
+    return [Call(wl, bh, dev, device, fused_hist=fused_hist)]
 
 
-def sub_record(wl, args, rank, world, device, peaks) -> dict:
+def sub_record(wl, args, rank, world, device, peaks, fused_hist=False) -> dict:
     """A full-size workload timed like the headline, with device-drawn inputs."""
     import torch
-    calls = device_calls(wl, device, rank_seed(rank))
+    calls = device_calls(wl, device, rank_seed(rank), fused_hist)
     sub_args = argparse.Namespace(**{**vars(args), "warmup": max(3, args.warmup)})
     with ClockSampler(_smi_index(device.index or 0)) as clk:
         res = time_calls(calls, sub_args, world, device, clk)
@@ -400,7 +411,8 @@ def sub_record(wl, args, rank, world, device, peaks) -> dict:
            "ms_per_step": res["ms_per_step"], "steps": sub_args.steps, "warmup": sub_args.warmup,
            "calls_per_step": len(calls), "queries_per_step": T, "config": config_of(wl, args),
            "roofline": r["roofline"], "stages": r["stages"], "gpu_launches": res["launches"],
-           "clocks": clk.summary(), "data": "synthetic, drawn on the device (seeded Philox)"}
+           "clocks": clk.summary(), "data": "synthetic, drawn on the device (seeded Philox)",
+           "indexer_topk": "fused through the emitted key histogram" if fused_hist else "unfused"}
     del calls
     torch.cuda.empty_cache()
     return rec
@@ -674,6 +686,9 @@ def main():
         for name in ("decode_b64", "decode_128k_mtp2", "decode_b1_128k", "chunked_64k"):
             if name != wl.name:
                 line["workloads"][name] = sub_record(WORKLOADS[name], args, rank, world, device, peaks)
+        # the indexer -> top-k fused through the emitted key histogram, same workload
+        line["workloads"]["decode_128k_mtp2_fused_hist"] = sub_record(WORKLOADS["decode_128k_mtp2"], args, rank,
+                                                                      world, device, peaks, fused_hist=True)
         line["workloads"]["project_append_4k"] = project_record(args, device, peaks, rank_seed(rank))
         torch.cuda.empty_cache()
 

@@ -172,6 +172,30 @@ dsa_status dsa_topk(const dsa_batch *batch, const float *scores, int64_t ld, int
                     void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Steps 2 -> 3 fused through a histogram ("四步工作流程" 第二步 索引器評分 feeding
+ * 第三步 Top-k 選擇): the indexer's epilogue also emits, per query row, the
+ * histogram of the top 11 bits of the order-preserving keys of its scores (the
+ * top-k's first radix pass), and the top-k takes it instead of computing it.
+ * The results are identical to dsa_indexer_scores + dsa_topk.
+ *   dsa_indexer_scores_hist: as dsa_indexer_scores, plus hist (device) uint32
+ *     [T, 2048] (zeroed and filled by the call).  Supported when the indexer's
+ *     query groups hold at most 4 tokens of at least 32 (padded) heads: every
+ *     H_I >= 36, and H_I in 20..32 with max_q_per_seq <= 4 (0: DSA_ERR_UNSUPPORTED).
+ *   dsa_topk_hist: as dsa_topk, plus hist (device) as emitted for the same
+ *     scores.  The clustered and the uncached top-k kernels skip their first pass
+ *     over the scores; the others ignore hist.
+ *   dsa_topk_uses_hist: 1 if dsa_topk_hist would use the histogram for this batch
+ *     (rows long or few enough for the clustered kernel, or longer than its
+ *     shared-memory cache), 0 otherwise (emitting it would then only cost time).
+ */
+dsa_status dsa_indexer_scores_hist(const dsa_batch *batch, const uint8_t *q_idx, const uint8_t *k_idx,
+                                   const float *w, int H_I, float *scores, int64_t ld, uint32_t *hist,
+                                   void *ws, size_t ws_bytes, void *stream);
+dsa_status dsa_topk_hist(const dsa_batch *batch, const float *scores, int64_t ld, const uint32_t *hist, int k,
+                         int32_t *idx, void *ws, size_t ws_bytes, void *stream);
+int dsa_topk_uses_hist(const dsa_batch *batch, int k);
+
+/*
  * Step 3, sparse MLA in MQA form ("四步工作流程" 第四步 執行稀疏 MLA; "DeepSeek-V3.2
  * 加速技术详解" 3.1 MQA版MLA and 3.2 hard selection).
  *   q   (device) bf16 bits [T, H, 576] query heads (latent part then RoPE part)

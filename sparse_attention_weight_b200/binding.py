@@ -25,7 +25,8 @@ OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_PROJECT = 0, 1, 2, 3, 4
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward",
            "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
-           "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout", "dsa_launch_count", "dsa_project_append")
+           "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout", "dsa_launch_count", "dsa_project_append",
+           "dsa_indexer_scores_hist", "dsa_topk_hist", "dsa_topk_uses_hist")
 NOALLOC_MAX_Q = 16384
 
 
@@ -67,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.dsa_forward.argtypes = [bp, vp, vp, vp, i32, vp, vp, i32, i32, f32, vp, vp, vp, sz, vp]
         L.dsa_indexer_scores_noalloc.argtypes = [bp, vp, vp, vp, i32, vp, i64, vp]
         L.dsa_project_append.argtypes = [bp, vp, vp, i32, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dsa_indexer_scores_hist.argtypes = [bp, vp, vp, vp, i32, vp, i64, vp, vp, sz, vp]
+        L.dsa_topk_hist.argtypes = [bp, vp, i64, vp, i32, vp, vp, sz, vp]
+        L.dsa_topk_uses_hist.argtypes = [bp, i32]
+        L.dsa_topk_uses_hist.restype = i32
         L.dsa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
         L.dsa_forward_ws_views.argtypes = [bp, i32, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(i64),
                                            ctypes.POINTER(vp)]
@@ -77,7 +82,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_launch_count.restype = ctypes.c_uint64
         for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward", "dsa_forward_ws_views",
                    "dsa_read_device_status", "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout",
-                   "dsa_project_append"):
+                   "dsa_project_append", "dsa_indexer_scores_hist", "dsa_topk_hist"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -176,6 +181,21 @@ def dsa_sparse_mla(batch: DeviceBatch, q, kv, idx, k: int, H: int, sm_scale: flo
     _check("dsa_sparse_mla", lib().dsa_sparse_mla(
         ctypes.byref(batch.struct), _ptr(q), _ptr(kv), _ptr(idx), k, H, sm_scale, _ptr(out), _ptr(lse), _ptr(ws),
         ws.numel(), _stream(stream)))
+
+
+def dsa_indexer_scores_hist(batch: DeviceBatch, q_idx, k_idx, w, H_I: int, scores, ld: int, hist, ws, stream=None):
+    _check("dsa_indexer_scores_hist", lib().dsa_indexer_scores_hist(
+        ctypes.byref(batch.struct), _ptr(q_idx), _ptr(k_idx), _ptr(w), H_I, _ptr(scores), ld, _ptr(hist), _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
+def dsa_topk_hist(batch: DeviceBatch, scores, ld: int, hist, k: int, idx, ws, stream=None):
+    _check("dsa_topk_hist", lib().dsa_topk_hist(ctypes.byref(batch.struct), _ptr(scores), ld, _ptr(hist), k,
+                                                _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def topk_uses_hist(batch: DeviceBatch, k: int) -> bool:
+    return bool(lib().dsa_topk_uses_hist(ctypes.byref(batch.struct), k))
 
 
 def dsa_project_append(batch: DeviceBatch, hidden, w_all, d_model: int, H_I: int, H: int, rope_base: float, q_idx,

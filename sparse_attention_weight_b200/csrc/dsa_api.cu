@@ -85,6 +85,10 @@ int hi_pad(int H_I) {
   return p;
 }
 bool h_ok(int H) { return H >= 8 && H <= 128 && H % 8 == 0; }
+// The indexer emits per-row key histograms when its query groups hold at most
+// four tokens (one shared-memory histogram per token slot) of >= 32 padded heads.
+int indexer_group(const dsa_batch* b, int H_I);
+bool hist_supported(const dsa_batch* b, int H_I) { return hi_pad(H_I) >= 32 && indexer_group(b, H_I) <= 4; }
 bool k_ok(int k) { return k >= 1 && k <= 2048; }
 
 int64_t default_ld(const dsa_batch* b) { return (static_cast<int64_t>(b->max_kv_len) + 3) / 4 * 4; }
@@ -179,7 +183,7 @@ WsLayout layout(void* ws, int op, const dsa_batch* b, int H, int k, int64_t ld) 
 dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
 dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* k_idx, const float* w, int H_I,
-                       float* scores, int64_t ld, const WsLayout& L, cudaStream_t st) {
+                       float* scores, int64_t ld, const WsLayout& L, cudaStream_t st, uint32_t* hist = nullptr) {
   if (b->num_q == 0) return DSA_OK;
   const int G = indexer_group(b, H_I);
   const int hp = hi_pad(H_I);
@@ -205,6 +209,7 @@ dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* 
   p.page_size = b->page_size;
   p.pages_per_seq = b->pages_per_seq;
   p.kv_rows = b->kv_rows;
+  p.hist = hist;
   int32_t* plan = L.plan;
   p.group_q0 = plan;
   p.group_cnt = plan + T;
@@ -222,9 +227,10 @@ dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* 
 }
 
 dsa_status run_topk(const dsa_batch* b, const float* scores, int64_t ld, int k, int32_t* idx, const WsLayout& L,
-                    cudaStream_t st) {
+                    cudaStream_t st, const uint32_t* hist = nullptr) {
   TopkParams p{};
   p.scores = scores;
+  p.hist = hist;
   p.ld = ld;
   p.idx = idx;
   p.k = k;
@@ -317,6 +323,45 @@ dsa_status dsa_topk(const dsa_batch* batch, const float* scores, int64_t ld, int
   return run_topk(batch, scores, ld, k, idx, L, st);
 }
 
+dsa_status dsa_indexer_scores_hist(const dsa_batch* batch, const uint8_t* q_idx, const uint8_t* k_idx, const float* w,
+                                   int H_I, float* scores, int64_t ld, uint32_t* hist, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!q_idx || !k_idx || !w || !scores || !hist)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!hi_ok(H_I) || !paging_ok(batch) || !hist_supported(batch, H_I)) return DSA_ERR_UNSUPPORTED;
+  if (ld < batch->max_kv_len || ld % 4 != 0) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(scores) || !aligned16(hist) ||
+      !aligned16(ws))
+    return DSA_ERR_UNSUPPORTED;
+  const WsLayout L = layout(ws, DSA_OP_INDEXER, batch, 8, 1, ld);
+  if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (batch->num_q > 0 &&
+      cudaMemsetAsync(hist, 0, static_cast<size_t>(batch->num_q) * 2048 * sizeof(uint32_t), st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return run_indexer(batch, q_idx, k_idx, w, H_I, scores, ld, L, st, hist);
+}
+
+dsa_status dsa_topk_hist(const dsa_batch* batch, const float* scores, int64_t ld, const uint32_t* hist, int k,
+                         int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!scores || !idx || !hist)) return DSA_ERR_INVALID_ARGUMENT;
+  if (!k_ok(k)) return DSA_ERR_UNSUPPORTED;
+  if (ld < batch->max_kv_len || ld % 4 != 0) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(scores) || !aligned16(hist) || !aligned16(ws)) return DSA_ERR_UNSUPPORTED;
+  const WsLayout L = layout(ws, DSA_OP_TOPK, batch, 8, k, ld);
+  if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  return run_topk(batch, scores, ld, k, idx, L, st, hist);
+}
+
+int dsa_topk_uses_hist(const dsa_batch* batch, int k) {
+  if (!batch_ok(batch) || !k_ok(k)) return 0;
+  return topk_uses_hist(batch->max_kv_len, batch->num_q, num_sms()) ? 1 : 0;
+}
+
 dsa_status dsa_sparse_mla(const dsa_batch* batch, const uint16_t* q, const uint16_t* kv, const int32_t* idx, int k,
                           int H, float sm_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
                           void* stream) {
@@ -345,6 +390,9 @@ dsa_status dsa_forward(const dsa_batch* batch, const uint8_t* q_idx, const uint8
   if (ws_bytes < L.bytes) return DSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  // The unfused indexer -> top-k: emitting the key histograms costs the
+  // indexer's epilogue more than skipping the first pass saves the top-k, which
+  // already reads each row once (measured; see dsa_indexer_scores_hist).
   dsa_status s = run_indexer(batch, q_idx, k_idx, w, H_I, L.scores, ld, L, st);
   if (s != DSA_OK) return s;
   s = run_topk(batch, L.scores, ld, k, L.idx, L, st);

@@ -353,6 +353,15 @@ __host__ __device__ __forceinline__ uint32_t sw128(uint32_t byte_off) {
   return byte_off ^ (((byte_off >> 7) & 7u) << 4);
 }
 
+// Order-preserving 32-bit key of an fp32 score (larger score = larger key;
+// -0.0 and +0.0 map to the same key).  The top-k selects on these keys; the
+// indexer's histogram of their top bits feeds its first radix pass.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  uint32_t b = __float_as_uint(x);
+  if ((b & 0x7fffffffu) == 0) b = 0;     // -0.0 == +0.0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
 // Register reallocation between warpgroups (all four warps of a warpgroup
 // execute the same instruction).  An increase waits until other warpgroups have
 // released enough of the registers the CTA was launched with.

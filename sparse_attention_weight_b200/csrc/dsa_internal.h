@@ -20,6 +20,7 @@ struct IndexerParams {
   int page_size;             // 0 = contiguous rows from kv_offset
   int pages_per_seq;
   int64_t kv_rows;           // rows of the k_idx buffer
+  uint32_t* hist;            // [T, 2048] histogram of the top 11 key bits per row (zeroed), or null
   // plan (workspace)
   int32_t* group_q0;         // [T]
   int32_t* group_cnt;        // [T]
@@ -37,6 +38,7 @@ struct IndexerParams {
 
 struct TopkParams {
   const float* scores;       // [T, ld]
+  const uint32_t* hist;      // [T, 2048] per-row histogram of the top 11 key bits, or null
   int64_t ld;
   int32_t* idx;              // [T, k]
   int k;
@@ -109,6 +111,9 @@ size_t mla_smem_bytes();
 cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int hi_pad,
                            int T, int B, int64_t kv_rows, int num_sms, cudaStream_t stream);
 cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream);
+// Whether the top-k kernel chosen for these rows takes an emitted histogram as
+// its first radix pass (the clustered and the uncached streaming kernels).
+bool topk_uses_hist(int max_kv_len, int T, int sms);
 cudaError_t launch_sparse_mla(const MlaParams& p, const CUtensorMap& tm_q, cudaStream_t stream);
 
 }  // namespace dsa

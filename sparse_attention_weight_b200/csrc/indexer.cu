@@ -12,11 +12,12 @@
 // Keys sit in TMEM lanes, so the per-head ReLU, weighting and head sum of the
 // epilogue run along one thread's own columns with no cross-lane reduction,
 // and each warp stores 32 consecutive scores of a row (coalesced).
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2..9 epilogue (two warps per TMEM lane quadrant, splitting the
-// group's tokens).  The grid is persistent (one CTA per SM); each
-// CTA takes a contiguous range of work items so the resident query tile is
-// reused across the key tiles of its group.
+// Warp roles (576 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
+// issuer, warps 2..17 epilogue (four per TMEM lane quadrant, each taking every
+// fourth token of the group).  The grid is persistent (one CTA per SM); each CTA
+// takes a contiguous range of work items so the resident query tile is reused
+// across the key tiles of its group.  A key tile is loaded as two 64-key halves,
+// each from its own cache page when the cache is paged.
 #include <cstdio>
 
 #include "dsa_common.cuh"
@@ -36,12 +37,14 @@ constexpr int kQBytes = 256 * DSA_D_INDEX;           // 32 KB (N <= 256)
 
 struct __align__(8) IdxSmem {
   uint8_t q[2][kQBytes];               // 1024-aligned (offset 0): query tiles of two groups
+  uint32_t hist[4][2048];              // per token slot of a group (G <= 4): histogram of the top 11 key bits
   uint8_t k[kStages][kTileBytes];      // 1024-aligned
   float w[kEpiWarps][256];             // per epilogue warp: head weights of the group
   int32_t n_vis[kEpiWarps][64];        // per epilogue warp: visible keys per token (G <= 64)
   uint64_t k_full[kStages], k_empty[kStages];
   uint64_t q_full[2], q_empty[2];
   uint64_t acc_full[kMaxAcc], acc_empty[kMaxAcc];
+  uint64_t hist_bar[4];                // per token slot: its four epilogue warps meet to flush
   uint64_t done;
   uint32_t tmem_base;
   int abort_flag;
@@ -81,6 +84,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int s = 0; s < kStages; ++s) { mbar_init(&S.k_full[s], 1); mbar_init(&S.k_empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&S.q_full[b], 1); mbar_init(&S.q_empty[b], 1); }
     for (int a = 0; a < kMaxAcc; ++a) { mbar_init(&S.acc_full[a], 1); mbar_init(&S.acc_empty[a], 32 * kEpiWarps); }
+    for (int h = 0; h < 4; ++h) mbar_init(&S.hist_bar[h], 4);
     mbar_init(&S.done, 1);
     S.abort_flag = 0;
     fence_mbar_init();
@@ -94,6 +98,8 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       reinterpret_cast<uint4*>(S.q)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
+  if (p.hist)
+    for (int i = threadIdx.x; i < 4 * 2048; i += blockDim.x) (&S.hist[0][0])[i] = 0u;
   if (warp == 1) tmem_alloc(&S.tmem_base, 512);
   tc_fence_before();
   __syncthreads();
@@ -219,10 +225,42 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       int prev_g = -1, cnt = 0, q0 = 0;
       int a = 0;                                  // accumulator buffer and its phase, advanced per item
       uint32_t aph = 0;
+      // Histogram emission (p.hist set; groups of at most 4 tokens, so token slot =
+      // tsub): the four warps of a token slot count the top 11 key bits of the
+      // group's scores in shared memory; when the group ends they meet, each adds
+      // a quarter of the bins to the row's global histogram, and meet again.
+      uint32_t nh = 0;                            // completed phases of hist_bar[tsub]
+      auto hsync = [&]() -> bool {
+        __syncwarp();
+        int ok = 1;
+        if (lane == 0) {
+          mbar_arrive(&S.hist_bar[tsub]);
+          ok = mbar_wait(&S.hist_bar[tsub], nh & 1, p.status, abort_flag) ? 1 : 0;
+        }
+        ++nh;
+        return __shfl_sync(0xffffffffu, ok, 0) != 0;
+      };
+      auto flush = [&](int fq0, int fcnt) -> bool {
+        if (!hsync()) return false;
+        if (tsub < fcnt) {
+          uint32_t* hs = S.hist[tsub];
+          uint32_t* hg = p.hist + static_cast<int64_t>(fq0 + tsub) * 2048;
+          for (int b = quad * 512 + lane; b < quad * 512 + 512; b += 32) {
+            const uint32_t v = hs[b];
+            if (v) {
+              atomicAdd(hg + b, v);
+              hs[b] = 0u;
+            }
+          }
+        }
+        return hsync();
+      };
+      bool hist_ok = true;
       for (int i = i0; i < i1; ++i) {
         while (g_hi <= i) { ++g; g_lo = g_hi; g_hi = p.item_off[g + 1]; }
         const int kt = i - g_lo;
         if (g != prev_g) {
+          if (p.hist && prev_g >= 0 && !(hist_ok = flush(q0, cnt))) break;
           __syncwarp();
           q0 = p.group_q0[g];
           cnt = p.group_cnt[g];
@@ -287,7 +325,20 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             const float sum = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
                               ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
-            if (s < snv[tok]) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = sum;
+            const bool vis = s < snv[tok];
+            if (vis) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = sum;
+            if (p.hist) {
+              // warp-aggregated: lanes whose bins agree with the first lane's add once
+              const uint32_t bin = order_key(sum) >> 21;
+              const uint32_t inmask = __ballot_sync(0xffffffffu, vis);
+              if (inmask) {
+                const int leader = __ffs(inmask) - 1;
+                const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
+                const uint32_t same = __ballot_sync(0xffffffffu, vis && bin == b0);
+                if (lane == leader) atomicAdd(&S.hist[tsub][b0], static_cast<uint32_t>(__popc(same)));
+                if (vis && bin != b0) atomicAdd(&S.hist[tsub][bin], 1u);
+              }
+            }
           }
         } else {
           constexpr int TPC = 32 / HI;             // tokens per 32-column chunk
@@ -315,6 +366,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_arrive(&S.acc_empty[a]);
         if (++a == nacc) { a = 0; aph ^= 1; }
       }
+      if (p.hist && hist_ok && prev_g >= 0 && !*abort_flag) flush(q0, cnt);
     }
   }
 
@@ -457,6 +509,7 @@ __global__ void __launch_bounds__(kPlanThreads) indexer_plan_kernel(IndexerParam
 
 }  // namespace
 
+static_assert(sizeof(IdxSmem) + 1024 <= 232448, "indexer shared memory exceeds the 227 KB per-CTA limit");
 size_t indexer_smem_bytes() { return sizeof(IdxSmem) + 1024; }
 
 // hi_pad: the token column stride (a power of two, 4..64); p.hi <= hi_pad is H_I.

@@ -30,12 +30,6 @@ constexpr int kCacheMax = 32768;         // keys cached in shared memory at most
 constexpr int kClusterMinLen = 8192;     // rows at least this long may share a cluster of CTAs
 constexpr int kClusterSegMax = 20480;    // keys cached per CTA of a cluster (80 KB: two CTAs per SM)
 
-__device__ __forceinline__ uint32_t order_key(float x) {
-  uint32_t b = __float_as_uint(x);
-  if ((b & 0x7fffffffu) == 0) b = 0;     // -0.0 == +0.0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
 struct Ctx {
   const float* row;
   uint32_t* cache;     // null when the row is not cached
@@ -178,16 +172,22 @@ __device__ __forceinline__ int row_length(const TopkParams& p, int t, int32_t* o
 
 // Exact top-k of row c (n > k) by three histogram passes (11, 11, 10 key bits)
 // and one output pass over the row: from the shared-memory cache when c.cache
-// is set (the first pass fills it), from L2 otherwise.
+// is set (the first pass fills it), from L2 otherwise.  An uncached row whose
+// first histogram the indexer already emitted (hist_in) skips the first pass.
 __device__ void select_streaming(const Ctx& c, int k, int32_t* out, uint32_t* hist, uint32_t* scratch,
-                                 uint32_t* sel) {
+                                 uint32_t* sel, const uint32_t* hist_in) {
   const bool cached = c.cache != nullptr;
   const int n = c.n;
   // pass 1: bits 31..21
-  for (int b = threadIdx.x; b < 2048; b += kThreads) hist[b] = 0;
-  __syncthreads();
-  hist_pass(c, false, cached, hist, 21, 11, 32, 0);
-  __syncthreads();
+  if (hist_in && !cached) {
+    for (int b = threadIdx.x; b < 2048; b += kThreads) hist[b] = __ldg(hist_in + b);
+    __syncthreads();
+  } else {
+    for (int b = threadIdx.x; b < 2048; b += kThreads) hist[b] = 0;
+    __syncthreads();
+    hist_pass(c, false, cached, hist, 21, 11, 32, 0);
+    __syncthreads();
+  }
   find_bin(hist, 2048, static_cast<uint32_t>(k), scratch, &sel[0], &sel[1]);
   const uint32_t b1 = sel[0], r1 = sel[1];
   __syncthreads();
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p, int cache_
   const int n = row_length(p, t, out);
   if (n <= 0) return;
   const Ctx c{p.scores + static_cast<int64_t>(t) * p.ld, n <= cache_elems ? cache : nullptr, n};
-  select_streaming(c, p.k, out, hist, scratch, sel);
+  select_streaming(c, p.k, out, hist, scratch, sel, p.hist ? p.hist + static_cast<int64_t>(t) * 2048 : nullptr);
 }
 
 // ---------------------------------------------------------------- long rows
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(TopkParams p) {
   const uint32_t m_total = (static_cast<uint32_t>(k) - r1) + hist[b1];   // keys at or above bin b1
   __syncthreads();
   if (m_total > static_cast<uint32_t>(kListCap)) {    // block-uniform: fall back to streaming
-    select_streaming(c, k, out, hist, scratch, sel);
+    select_streaming(c, k, out, hist, scratch, sel, nullptr);
     return;
   }
 
@@ -501,8 +501,9 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, in
   __syncthreads();
   cl_sync();                                               // every copy is cleared before any reduction
 
-  // pass 1: cache the segment's keys and histogram bits 31..21; four 16-byte
-  // loads per thread in flight
+  // pass 1: cache the segment's keys and histogram bits 31..21 (unless the
+  // indexer emitted the row's histogram); four 16-byte loads per thread in flight
+  const bool have_hist = p.hist != nullptr;               // uniform over the grid
   constexpr int kUnroll = 4;
   for (int base = 0; base < m; base += kStep * kUnroll) {
     uint32_t kk[kUnroll][kPer];
@@ -521,15 +522,22 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, in
     for (int w = 0; w < kUnroll; ++w) {
       const int i = base + w * kStep + threadIdx.x * kPer;
       if (i < m) *reinterpret_cast<uint4*>(cache + i) = make_uint4(kk[w][0], kk[w][1], kk[w][2], kk[w][3]);
+      if (!have_hist) {
 #pragma unroll
-      for (int u = 0; u < kPer; ++u) {
-        hist_add(S.local, kk[w][u] >> 21, (i + u) < m, lane);
+        for (int u = 0; u < kPer; ++u) hist_add(S.local, kk[w][u] >> 21, (i + u) < m, lane);
       }
     }
   }
   __syncthreads();
-  cl_push(S, S.global[0], 2048, C);
-  cl_sync();                                               // the cluster's histogram is complete everywhere
+  if (have_hist) {
+    // every CTA of the cluster reads the same row histogram: no reduction needed
+    const uint32_t* hg = p.hist + static_cast<int64_t>(t) * 2048;
+    for (int b = threadIdx.x; b < 2048; b += kThreads) S.global[0][b] = __ldg(hg + b);
+    __syncthreads();
+  } else {
+    cl_push(S, S.global[0], 2048, C);
+    cl_sync();                                             // the cluster's histogram is complete everywhere
+  }
   find_bin(S.global[0], 2048, static_cast<uint32_t>(k), S.scratch, &S.sel[0], &S.sel[1]);
   const uint32_t b1 = S.sel[0], r1 = S.sel[1];
   __syncthreads();
@@ -623,6 +631,29 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, in
 }
 
 }  // namespace
+
+// Which kernel launch_topk picks for these rows: 2..8 = a cluster of that many
+// CTAs per row, 1 = the two-read long-row kernel, 0 = the streaming kernel with
+// rows cached in shared memory, -1 = the streaming kernel reading rows from L2.
+int topk_plan(int max_kv_len, int T, int sms) {
+  if (max_kv_len >= kClusterMinLen) {
+    auto seg_of = [&](int c) { return (((max_kv_len + c - 1) / c + kStep - 1) / kStep) * kStep; };
+    int c_fit = 1;
+    while (c_fit <= 8 && seg_of(c_fit) > kClusterSegMax) c_fit <<= 1;
+    int c_par = 8;
+    while (c_par > 1 && T * c_par > 2 * sms) c_par >>= 1;
+    const int C = c_fit > c_par ? c_fit : c_par;
+    if (C >= 2 && C <= 8) return C;
+  }
+  const int cache_elems = ((max_kv_len + kStep - 1) / kStep) * kStep;
+  if (cache_elems > kCacheMax && T <= 2 * sms) return 1;
+  return cache_elems > kCacheMax ? -1 : 0;
+}
+
+bool topk_uses_hist(int max_kv_len, int T, int sms) {
+  const int plan = topk_plan(max_kv_len, T, sms);
+  return plan >= 2 || plan == -1;
+}
 
 cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;

@@ -128,6 +128,26 @@ def test_project_append_host_checks(lib):
     assert call(ws_bytes=1024) == 3
 
 
+def test_histogram_fusion_host_checks(lib):
+    """dsa_indexer_scores_hist needs groups of <= 4 tokens of >= 32 padded heads;
+    dsa_topk_uses_hist follows the top-k's kernel choice."""
+    ws, p, big = 0x50000, 0x60000, 1 << 40
+    b = _fake_batch()                                   # 16 queries, max_q_per_seq 0 (taken as 16)
+    call = lambda bb, hi, hist=p: lib.dsa_indexer_scores_hist(ctypes.byref(bb), p, p, p, hi, p, 3000, hist, ws,
+                                                              big if hist else 0, None)
+    assert call(b, 64, hist=0) == 1                     # no histogram buffer
+    assert call(b, 16) == 2                             # 16 heads: below 32 padded heads
+    assert call(b, 32) == 2                             # 32 heads, 16 queries per sequence: groups of 8
+    b4 = B.DsaBatch(2, 16, 3000, 4, 6000, 0x10000, 0x20000, 0x30000, 0x40000)
+    assert call(b4, 32, hist=p + 4) == 2                # alignment of the histogram
+    assert lib.dsa_topk_hist(ctypes.byref(b), p, 3000, 0, 2048, p, ws, big, None) == 1
+    long_few = B.DsaBatch(16, 16, 131072, 1, 16 * 131072, 0x10000, 0x20000, 0x30000, 0x40000)
+    short_many = B.DsaBatch(1, 8192, 8192, 8192, 8192, 0x10000, 0x20000, 0x30000, 0x40000)
+    assert lib.dsa_topk_uses_hist(ctypes.byref(long_few), 2048) == 1      # clustered rows
+    assert lib.dsa_topk_uses_hist(ctypes.byref(short_many), 2048) == 0    # rows cached per CTA
+    assert lib.dsa_topk_uses_hist(None, 2048) == 0
+
+
 def test_read_device_status_rejects_null(lib):
     flags = ctypes.c_uint32()
     assert lib.dsa_read_device_status(None, ctypes.byref(flags), None) == 1
