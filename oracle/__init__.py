@@ -7,3 +7,4 @@ from .dsa_ref import (attention_probs, bf16_decode, bf16_encode_rne, dense_mla, 
                       e4m3_decode, e4m3_encode_rne, forward, indexer_scores, sparse_mla,
                       topk_select)
 from . import projection  # noqa: F401,E402
+from . import backward  # noqa: F401,E402
