@@ -30,9 +30,14 @@ import numpy as np
 
 
 def sparse_mla_backward(q: np.ndarray, kv: np.ndarray, idx: np.ndarray, sm_scale: float, d_out: np.ndarray,
-                        d_v: int = 512):
+                        d_v: int = 512, out=None, lse=None):
     """q: [T, H, 576], kv: [S, 576], idx: [T, k] (-1 unused), d_out: [T, H, d_v]
-    (all float64).  Returns (dq [T, H, 576], dkv [S, 576])."""
+    (all float64).  Returns (dq [T, H, 576], dkv [S, 576]).
+
+    With `out` [T, H, d_v] and `lse` [T, H] given (a forward's stored output and
+    log-sum-exp), D is formed from that output and p from that lse, as a backward
+    that keeps only the forward's outputs does; without them both are recomputed
+    exactly."""
     T, H, D = q.shape
     dq = np.zeros_like(q, dtype=np.float64)
     dkv = np.zeros((kv.shape[0], D), dtype=np.float64)
@@ -43,9 +48,12 @@ def sparse_mla_backward(q: np.ndarray, kv: np.ndarray, idx: np.ndarray, sm_scale
         sel = idx[t][pos].astype(np.int64)
         rows = kv[sel]                                  # [m, 576]
         z = sm_scale * (q[t] @ rows.T)                  # [H, m]
-        e = np.exp(z - z.max(axis=1, keepdims=True))
-        p = e / e.sum(axis=1, keepdims=True)
-        o = p @ rows[:, :d_v]                           # [H, d_v]
+        if lse is None:
+            e = np.exp(z - z.max(axis=1, keepdims=True))
+            p = e / e.sum(axis=1, keepdims=True)
+        else:
+            p = np.exp(z - np.asarray(lse[t], dtype=np.float64)[:, None])
+        o = p @ rows[:, :d_v] if out is None else np.asarray(out[t], dtype=np.float64)   # [H, d_v]
         dP = d_out[t] @ rows[:, :d_v].T                 # [H, m]
         Dh = np.sum(d_out[t] * o, axis=1, keepdims=True)
         dZ = p * (dP - Dh)                              # [H, m]

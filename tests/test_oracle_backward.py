@@ -72,3 +72,12 @@ def test_unselected_rows_get_no_gradient_and_identical_rows_give_no_query_gradie
     same = np.where(idx >= 0, 4, -1)
     dq2, _ = BW.sparse_mla_backward(q, kv, same, 0.1, dout)
     assert np.abs(dq2).max() <= 1e-12 * np.abs(dq).max()
+
+
+def test_stored_forward_outputs_reproduce_the_exact_gradient():
+    q, kv, idx, dout = _case(seed=4)
+    scale = 0.05
+    out, lse = oracle.sparse_mla(q, kv, idx, scale)
+    a = BW.sparse_mla_backward(q, kv, idx, scale, dout)
+    b = BW.sparse_mla_backward(q, kv, idx, scale, dout, out=out, lse=lse)
+    assert np.allclose(a[0], b[0], rtol=1e-12, atol=1e-14) and np.allclose(a[1], b[1], rtol=1e-12, atol=1e-14)
