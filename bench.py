@@ -474,6 +474,67 @@ def project_record(args, device, peaks, seed: int) -> dict:
                     "RoPE / casts / append by the library's own kernel"}
 
 
+def backward_record(args, device, peaks, seed: int) -> dict:
+    """The sparse-MLA backward (dsa_sparse_mla_backward) on a 2048-token prefill
+    (k = 2048, H = 128: every query attends over all its visible rows), after a
+    forward call that provides the stored output and lse."""
+    import torch
+
+    from sparse_attention_weight_b200 import binding as B
+    from sparse_attention_weight_b200 import inputs
+    L, k, H = 2048, 2048, 128
+    wl = dataclasses.replace(WORKLOADS["prefill_8k"], name="prefill_2k_bwd", seq_len=L, k=k, heads=H)
+    bh = inputs.make_batch(wl, seed)
+    dev = {**inputs.device_query_tensors(wl, bh, device, seed), **inputs.device_cache_tensors(wl, bh, device, seed)}
+    db = B.DeviceBatch.from_host(bh, device)
+    idx = torch.full((L, k), -1, dtype=torch.int32, device=device)
+    ar = torch.arange(k, device=device, dtype=torch.int32)
+    for t0 in range(0, L, 256):                                 # query t selects rows 0..t
+        tt = torch.arange(t0, min(L, t0 + 256), device=device, dtype=torch.int32)[:, None]
+        idx[t0:t0 + tt.shape[0]] = torch.where(ar[None, :] <= tt, ar[None, :], torch.full_like(ar[None, :], -1))
+    out = torch.empty((L, H, D_V), dtype=torch.int16, device=device)
+    lse = torch.empty((L, H), dtype=torch.float32, device=device)
+    ws = B.workspace(B.OP_SPARSE_MLA, db, H=H, k=k, device=device)
+    B.dsa_sparse_mla(db, dev["q"], dev["kv"], idx, k, H, wl.sm_scale, out, lse, ws)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed * 31 + 5)
+    dout = torch.randn((L, H, D_V), generator=g, device=device).to(torch.bfloat16).view(torch.int16)
+    dq = torch.empty((L, H, D_QK), dtype=torch.float32, device=device)
+    dkv = torch.zeros((L, D_QK), dtype=torch.float32, device=device)
+    wsb = B.workspace(B.OP_MLA_BACKWARD, db, H=H, k=k, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    run = lambda: B.dsa_sparse_mla_backward(db, dev["q"], dev["kv"], idx, k, H, wl.sm_scale, out, lse, dout, dq,
+                                             dkv, wsb)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        dkv.zero_()
+        run()
+    torch.cuda.synchronize()
+    if B.read_device_status(wsb):
+        raise RuntimeError("device status flags in dsa_sparse_mla_backward")
+    steps = max(3, min(args.steps, 5))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    l0 = B.launch_count()
+    for e0, e1 in ev:
+        flush.zero_()
+        dkv.zero_()
+        e0.record()
+        run()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+    pairs = L * (L + 1) // 2
+    flop = pairs * H * 2 * (2 * D_QK + D_V + D_QK + D_V)      # z, dP, dQ, dK, dV per (query, row, head)
+    return {"metric": "sparse-MLA backward tokens/s", "value": L / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": steps, "calls_per_step": 1, "queries_per_step": L,
+            "config": {"workload": "prefill_2k_bwd", "seq_len": L, "k": k, "heads": H, "selected_pairs": pairs,
+                       "l2": "flushed before every timed step (512 MB write)"},
+            "stages": {"mla_backward": {"ms": ms, "tflops": flop / (ms / 1e3) / 1e12,
+                                        "frac_of_bf16_tensor_peak": flop / (ms / 1e3) / 1e12 / peaks["bf16"]}},
+            "gpu_launches": B.launch_count() - l0,
+            "data": "synthetic, drawn on the device (seeded Philox); fp32 CUDA-core kernel with atomic d_kv"}
+
+
 def config_of(wl, args) -> dict:
     decode = wl.kind == "decode"
     return {"workload": wl.name, "k": wl.k, "h_index": wl.h_index, "heads": wl.heads, "d_qk": D_QK, "d_v": D_V,
@@ -690,6 +751,7 @@ def main():
         line["workloads"]["decode_128k_mtp2_fused_hist"] = sub_record(WORKLOADS["decode_128k_mtp2"], args, rank,
                                                                       world, device, peaks, fused_hist=True)
         line["workloads"]["project_append_4k"] = project_record(args, device, peaks, rank_seed(rank))
+        line["workloads"]["prefill_2k_bwd"] = backward_record(args, device, peaks, rank_seed(rank))
         torch.cuda.empty_cache()
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

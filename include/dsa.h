@@ -97,6 +97,7 @@ typedef struct dsa_batch {
 #define DSA_OP_SPARSE_MLA 2
 #define DSA_OP_FORWARD 3
 #define DSA_OP_PROJECT 4
+#define DSA_OP_MLA_BACKWARD 5
 
 /*
  * Bytes of workspace `ws` an operation needs (always >= 256: the status word and
@@ -194,6 +195,31 @@ dsa_status dsa_indexer_scores_hist(const dsa_batch *batch, const uint8_t *q_idx,
 dsa_status dsa_topk_hist(const dsa_batch *batch, const float *scores, int64_t ld, const uint32_t *hist, int k,
                          int32_t *idx, void *ws, size_t ws_bytes, void *stream);
 int dsa_topk_uses_hist(const dsa_batch *batch, int k);
+
+/*
+ * Backward of step 3 (sparse continued training, "DeepSeek-V3.2加速技术详解" §04:
+ * the model learns through the selected tokens only): gradients of the sparse MLA
+ * output with respect to the queries and the latent cache rows, for an output
+ * gradient d_out, with the selection held fixed (no gradient through top-k).
+ * For query t, head h and selected entries i (cache rows r_i):
+ *   z_i = sm_scale q.kv_i, p_i = exp(z_i - lse), D = d_out.out, dZ_i = p_i (d_out.kv_i[:512] - D)
+ *   d_q[t,h]  = sm_scale sum_i dZ_i kv_i
+ *   d_kv[r_i] += sm_scale dZ_i q[t,h] + p_i [d_out[t,h], 0]
+ *   q, kv, idx, k, H, sm_scale: as in dsa_sparse_mla (the same call's inputs)
+ *   out, lse (device) the forward's bf16 output and fp32 log-sum-exp (lse required)
+ *   d_out (device) bf16 bits [T, H, 512]
+ *   d_q   (device) fp32 [T, H, 576], written
+ *   d_kv  (device) fp32 [kv_rows, 576]: ADDED to (atomically; a row selected by
+ *         several queries or entries receives every contribution).  The caller
+ *         zeroes it before the first call of a step.  Summation order varies from
+ *         run to run (atomics), so d_kv is reproducible to rounding only.
+ * Workspace: dsa_workspace_size(DSA_OP_MLA_BACKWARD, ...) (the status word).
+ * Supported: as dsa_sparse_mla; d_q and d_kv 16-byte aligned.
+ */
+dsa_status dsa_sparse_mla_backward(const dsa_batch *batch, const uint16_t *q, const uint16_t *kv, const int32_t *idx,
+                                   int k, int H, float sm_scale, const uint16_t *out, const float *lse,
+                                   const uint16_t *d_out, float *d_q, float *d_kv, void *ws, size_t ws_bytes,
+                                   void *stream);
 
 /*
  * Step 3, sparse MLA in MQA form ("四步工作流程" 第四步 執行稀疏 MLA; "DeepSeek-V3.2

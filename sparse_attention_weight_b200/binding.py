@@ -21,12 +21,12 @@ DSA_OK = 0
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARGUMENT", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_WORKSPACE_TOO_SMALL", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_DEVICE"}
 DEV_BAD_QUERY, DEV_BAD_INDEX, DEV_TIMEOUT = 1, 2, 4
-OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_PROJECT = 0, 1, 2, 3, 4
+OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_PROJECT, OP_MLA_BACKWARD = 0, 1, 2, 3, 4, 5
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward",
            "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
            "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout", "dsa_launch_count", "dsa_project_append",
-           "dsa_indexer_scores_hist", "dsa_topk_hist", "dsa_topk_uses_hist")
+           "dsa_indexer_scores_hist", "dsa_topk_hist", "dsa_topk_uses_hist", "dsa_sparse_mla_backward")
 NOALLOC_MAX_Q = 16384
 
 
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_indexer_scores_hist.argtypes = [bp, vp, vp, vp, i32, vp, i64, vp, vp, sz, vp]
         L.dsa_topk_hist.argtypes = [bp, vp, i64, vp, i32, vp, vp, sz, vp]
         L.dsa_topk_uses_hist.argtypes = [bp, i32]
+        L.dsa_sparse_mla_backward.argtypes = [bp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
         L.dsa_topk_uses_hist.restype = i32
         L.dsa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
         L.dsa_forward_ws_views.argtypes = [bp, i32, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(i64),
@@ -82,7 +83,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_launch_count.restype = ctypes.c_uint64
         for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward", "dsa_forward_ws_views",
                    "dsa_read_device_status", "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout",
-                   "dsa_project_append", "dsa_indexer_scores_hist", "dsa_topk_hist"):
+                   "dsa_project_append", "dsa_indexer_scores_hist", "dsa_topk_hist", "dsa_sparse_mla_backward"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -192,6 +193,13 @@ def dsa_indexer_scores_hist(batch: DeviceBatch, q_idx, k_idx, w, H_I: int, score
 def dsa_topk_hist(batch: DeviceBatch, scores, ld: int, hist, k: int, idx, ws, stream=None):
     _check("dsa_topk_hist", lib().dsa_topk_hist(ctypes.byref(batch.struct), _ptr(scores), ld, _ptr(hist), k,
                                                 _ptr(idx), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def dsa_sparse_mla_backward(batch: DeviceBatch, q, kv, idx, k: int, H: int, sm_scale: float, out, lse, d_out, d_q,
+                            d_kv, ws, stream=None):
+    _check("dsa_sparse_mla_backward", lib().dsa_sparse_mla_backward(
+        ctypes.byref(batch.struct), _ptr(q), _ptr(kv), _ptr(idx), k, H, sm_scale, _ptr(out), _ptr(lse), _ptr(d_out),
+        _ptr(d_q), _ptr(d_kv), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def topk_uses_hist(batch: DeviceBatch, k: int) -> bool:

@@ -287,6 +287,7 @@ extern "C" {
 size_t dsa_workspace_size(int op, const dsa_batch* batch, int H_I, int H, int k, int64_t ld) {
   if (!batch_ok(batch)) return 0;
   if (op == DSA_OP_PROJECT) return hi_ok(H_I) && h_ok(H) ? proj_layout(nullptr, batch, H_I, H).bytes : 0;
+  if (op == DSA_OP_MLA_BACKWARD) return kWsHeader;
   if (op < DSA_OP_INDEXER || op > DSA_OP_FORWARD) return 0;
   if ((op == DSA_OP_SPARSE_MLA || op == DSA_OP_FORWARD) && (!h_ok(H) || !k_ok(k))) return 0;
   if (op == DSA_OP_FORWARD && !k_ok(k)) return 0;
@@ -355,6 +356,46 @@ dsa_status dsa_topk_hist(const dsa_batch* batch, const float* scores, int64_t ld
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(L.status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
   return run_topk(batch, scores, ld, k, idx, L, st, hist);
+}
+
+dsa_status dsa_sparse_mla_backward(const dsa_batch* batch, const uint16_t* q, const uint16_t* kv, const int32_t* idx,
+                                   int k, int H, float sm_scale, const uint16_t* out, const float* lse,
+                                   const uint16_t* d_out, float* d_q, float* d_kv, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  if (!batch_ok(batch) || !ws) return DSA_ERR_INVALID_ARGUMENT;
+  if (batch->num_q > 0 && (!q || !kv || !idx || !out || !lse || !d_out || !d_q || !d_kv))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!h_ok(H) || !k_ok(k) || !paging_ok(batch)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || !aligned16(d_out) || !aligned16(d_q) ||
+      !aligned16(d_kv) || !aligned16(ws))
+    return DSA_ERR_UNSUPPORTED;
+  if (ws_bytes < kWsHeader) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) != cudaSuccess) return DSA_ERR_CUDA;
+  MlaBwdParams p{};
+  p.q = q;
+  p.kv = kv;
+  p.idx = idx;
+  p.k = k;
+  p.H = H;
+  p.sm_scale = sm_scale;
+  p.out = out;
+  p.lse = lse;
+  p.d_out = d_out;
+  p.d_q = d_q;
+  p.d_kv = d_kv;
+  p.q_seq = batch->q_seq;
+  p.kv_offset = batch->kv_offset;
+  p.kv_len = batch->kv_len;
+  p.page_table = batch->page_table;
+  p.page_size = batch->page_size;
+  p.pages_per_seq = batch->pages_per_seq;
+  p.num_seqs = batch->num_seqs;
+  p.kv_rows = batch->kv_rows;
+  p.T = batch->num_q;
+  p.status = status;
+  return cuda_status(launch_mla_backward(p, st));
 }
 
 int dsa_topk_uses_hist(const dsa_batch* batch, int k) {

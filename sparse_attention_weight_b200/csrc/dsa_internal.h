@@ -100,6 +100,31 @@ struct ProjParams {
   uint32_t* status;
 };
 
+struct MlaBwdParams {
+  const uint16_t* q;         // [T, H, 576] bf16
+  const uint16_t* kv;        // [rows, 576] bf16
+  const int32_t* idx;        // [T, k]
+  int k;
+  int H;
+  float sm_scale;
+  const uint16_t* out;       // [T, H, 512] bf16, the forward's output
+  const float* lse;          // [T, H], the forward's log-sum-exp
+  const uint16_t* d_out;     // [T, H, 512] bf16
+  float* d_q;                // [T, H, 576]
+  float* d_kv;               // [rows, 576], accumulated
+  const int32_t* q_seq;
+  const int64_t* kv_offset;
+  const int32_t* kv_len;
+  const int32_t* page_table;
+  int page_size;
+  int pages_per_seq;
+  int num_seqs;
+  int64_t kv_rows;
+  int T;
+  uint32_t* status;
+};
+cudaError_t launch_mla_backward(const MlaBwdParams& p, cudaStream_t stream);
+
 // Counts kernel launches made by the library (dsa_launch_count).
 void count_launches(int n);
 
