@@ -37,7 +37,6 @@ constexpr int kQBytes = 256 * DSA_D_INDEX;           // 32 KB (N <= 256)
 
 struct __align__(8) IdxSmem {
   uint8_t q[2][kQBytes];               // 1024-aligned (offset 0): query tiles of two groups
-  uint32_t hist[4][2048];              // per token slot of a group (G <= 4): histogram of the top 11 key bits
   uint8_t k[kStages][kTileBytes];      // 1024-aligned
   float w[kEpiWarps][256];             // per epilogue warp: head weights of the group
   int32_t n_vis[kEpiWarps][64];        // per epilogue warp: visible keys per token (G <= 64)
@@ -48,6 +47,8 @@ struct __align__(8) IdxSmem {
   uint64_t done;
   uint32_t tmem_base;
   int abort_flag;
+  // last, so that a launch without histograms leaves it out of its allocation:
+  uint32_t hist[4][2048];              // per token slot of a group (G <= 4): histogram of the top 11 key bits
 };
 
 // Largest g with item_off[g] <= i (item_off is non-decreasing, item_off[0] = 0).
@@ -60,7 +61,9 @@ __device__ __forceinline__ int find_group(const int32_t* item_off, int ngroups, 
   return lo;
 }
 
-template <int HI>
+// HIST: the epilogue also emits the per-row key histograms (p.hist); a
+// compile-time switch, so that the plain indexer carries none of its code.
+template <int HI, bool HIST>
 __global__ void __launch_bounds__(kIdxThreads, 1)
 indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                IndexerParams p) {
@@ -98,7 +101,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       reinterpret_cast<uint4*>(S.q)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
-  if (p.hist)
+  if (HIST)
     for (int i = threadIdx.x; i < 4 * 2048; i += blockDim.x) (&S.hist[0][0])[i] = 0u;
   if (warp == 1) tmem_alloc(&S.tmem_base, 512);
   tc_fence_before();
@@ -260,7 +263,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         while (g_hi <= i) { ++g; g_lo = g_hi; g_hi = p.item_off[g + 1]; }
         const int kt = i - g_lo;
         if (g != prev_g) {
-          if (p.hist && prev_g >= 0 && !(hist_ok = flush(q0, cnt))) break;
+          if (HIST && prev_g >= 0 && !(hist_ok = flush(q0, cnt))) break;
           __syncwarp();
           q0 = p.group_q0[g];
           cnt = p.group_cnt[g];
@@ -327,7 +330,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                               ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
             const bool vis = s < snv[tok];
             if (vis) p.scores[static_cast<int64_t>(q0 + tok) * p.ld + s] = sum;
-            if (p.hist) {
+            if constexpr (HIST) {
               // warp-aggregated: lanes whose bins agree with the first lane's add once
               const uint32_t bin = order_key(sum) >> 21;
               const uint32_t inmask = __ballot_sync(0xffffffffu, vis);
@@ -366,7 +369,7 @@ indexer_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         mbar_arrive(&S.acc_empty[a]);
         if (++a == nacc) { a = 0; aph ^= 1; }
       }
-      if (p.hist && hist_ok && prev_g >= 0 && !*abort_flag) flush(q0, cnt);
+      if (HIST && hist_ok && prev_g >= 0 && !*abort_flag) flush(q0, cnt);
     }
   }
 
@@ -511,6 +514,10 @@ __global__ void __launch_bounds__(kPlanThreads) indexer_plan_kernel(IndexerParam
 
 static_assert(sizeof(IdxSmem) + 1024 <= 232448, "indexer shared memory exceeds the 227 KB per-CTA limit");
 size_t indexer_smem_bytes() { return sizeof(IdxSmem) + 1024; }
+// without histograms the trailing histogram array is not allocated
+static size_t indexer_smem_bytes_for(bool hist) {
+  return hist ? indexer_smem_bytes() : indexer_smem_bytes() - sizeof(uint32_t) * 4 * 2048;
+}
 
 // hi_pad: the token column stride (a power of two, 4..64); p.hi <= hi_pad is H_I.
 cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, const IndexerParams& p, int hi_pad,
@@ -519,7 +526,7 @@ cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, con
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   count_launches(1);
-  const size_t smem = indexer_smem_bytes();
+  const size_t smem = indexer_smem_bytes_for(p.hist != nullptr);
   auto launch = [&](auto kern) -> cudaError_t {
     cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
@@ -529,12 +536,19 @@ cudaError_t launch_indexer(const CUtensorMap& tm_q, const CUtensorMap& tm_k, con
     if (err == cudaSuccess) count_launches(1);
     return err;
   };
+  if (p.hist) {                        // the host allows histograms only with >= 32 padded heads
+    switch (hi_pad) {
+      case 32: return launch(indexer_kernel<32, true>);
+      case 64: return launch(indexer_kernel<64, true>);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (hi_pad) {
-    case 4: return launch(indexer_kernel<4>);
-    case 8: return launch(indexer_kernel<8>);
-    case 16: return launch(indexer_kernel<16>);
-    case 32: return launch(indexer_kernel<32>);
-    case 64: return launch(indexer_kernel<64>);
+    case 4: return launch(indexer_kernel<4, false>);
+    case 8: return launch(indexer_kernel<8, false>);
+    case 16: return launch(indexer_kernel<16, false>);
+    case 32: return launch(indexer_kernel<32, false>);
+    case 64: return launch(indexer_kernel<64, false>);
     default: return cudaErrorInvalidValue;
   }
 }
