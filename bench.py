@@ -53,12 +53,12 @@ from sparse_attention_weight_b200.configs import WORKLOADS  # noqa: E402
 L2_FLUSH_BYTES = 512 << 20
 D_QK, D_V, D_INDEX = 576, 512, 128
 # DRAM bytes (read + write) per query of the sparse-MLA kernel on prefill, from
-# one ncu capture of the kernel as it stands: dram__bytes_read.sum (361.36 MB) +
-# dram__bytes_write.sum (258.47 MB) of the timed launch of
+# one ncu capture of the kernel as it stands: dram__bytes_read.sum (361.41 MB) +
+# dram__bytes_write.sum (259.02 MB) of the timed launch of
 # `bench.py --seq-len 2304 --steps 1 --warmup 1 --no-e2e --no-cpu-baseline`,
 # divided by its 2304 queries (the traffic is the queries in and the outputs out;
 # the gathered cache rows hit L2).  None while no capture describes the kernel.
-MLA_TRAFFIC_BYTES_PER_QUERY = (361.357568e6 + 258.470656e6) / 2304
+MLA_TRAFFIC_BYTES_PER_QUERY = (361.408e6 + 259.017216e6) / 2304
 # Workloads run with a paged cache, and their page size (rows).
 PAGED = {"decode_b1_128k": 64}
 
