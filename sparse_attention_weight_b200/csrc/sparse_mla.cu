@@ -70,10 +70,10 @@ constexpr int kRoleWarp = 4 + kSWarps + kVWarps;   // first of the four single-l
 // Registers: launched at 80 per thread (768 x 80 = 61,440); the softmax
 // warpgroup takes 160, every other warpgroup gives back down to 64
 // (128 x 160 + 640 x 64 = 61,440).
-// Readers of a plan slot that release it (plan_free): the 128 softmax threads,
-// the 16 gather warps and three single-lane roles (plus the PV issuer in the
-// even CTA).
-constexpr uint32_t kPlanReaders = 128 + kSWarps + kVWarps + 3;
+// Readers of a plan slot that release it (plan_free), one arrival each: the 4
+// softmax warps, the 16 gather warps and three single-lane roles (plus the PV
+// issuer in the even CTA).
+constexpr uint32_t kPlanReaders = 4 + kSWarps + kVWarps + 3;
 constexpr uint32_t kLaunchRegs = 80;
 constexpr uint32_t kRegsSoftmax = 160;
 constexpr uint32_t kRegsOther = 64;
@@ -242,11 +242,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
       mbar_init(&S.v_full[i], 1); mbar_init(&S.v_empty[i], 1); mbar_init(&S.v_loaded[i], kVWarps * 32);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 4); mbar_init(&S.mx_bar[i], 128);
+      mbar_init(&S.s_ready[i], 1); mbar_init(&S.s_free[i], 4); mbar_init(&S.mx_bar[i], 4);
       mbar_init(&S.plan_ready[i], kSWarps); mbar_init(&S.plan_free[i], kPlanReaders + (rank == 0 ? 1 : 0));
     }
     for (int h = 0; h < 2; ++h) { mbar_init(&S.p_full[h], 2); mbar_init(&S.p_empty[h], 1); }
-    mbar_init(&S.l_bar, 128);
+    mbar_init(&S.l_bar, 4);
     mbar_init(&S.o_done[0], 1); mbar_init(&S.o_done[1], 1);
     mbar_init(&S.o_full, 1);
     mbar_init(&S.o_free, 4);
@@ -302,7 +302,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
             if (half == 0) p.part_lse[(static_cast<int64_t>(I.t) * p.splits + I.split) * H + h] = -INFINITY;
           }
         }
-        mbar_arrive(&S.plan_free[b]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.plan_free[b]);
         continue;
       }
       float m_ref = -INFINITY, l = 0.f;
@@ -329,7 +330,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         }
         // pair maximum of this head over the whole block
         S.xmax[sb][tid] = mloc;
-        mbar_arrive(&S.mx_bar[sb]);
+        __syncwarp();                                      // one arrival per warp (count 4)
+        if (lane == 0) mbar_arrive(&S.mx_bar[sb]);
         if (!warp_wait(&S.mx_bar[sb], sph, p.status, ab, false)) { ok = false; break; }
         const float mblk = fmaxf(mloc, S.xmax[sb][tid ^ 64]);
         const bool rescale = mblk > m_ref + kRescaleThreshold;
@@ -427,14 +429,16 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap tm_q, MlaParams p) {
         // carries the odd CTA's 8 bytes)
         if (lane == 0) pair_signal(rank, &S.p_full[half], &S.mbox_pfull[half][warp & 1], (warp & 1) == 0, 8);
       }
-      mbar_arrive(&S.plan_free[b]);                       // this query's validity words are no longer read
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.plan_free[b]);       // this query's validity words are no longer read
       if (!ok) break;
       // ---- epilogue: wait for the last PV, combine the two row halves, write out,
       // then release O to the PV MMAs of the next query
       if (!warp_wait(&S.o_full, ne & 1, p.status, ab, false)) break;
       tc_fence_after();
       S.lsum[tid] = l;
-      mbar_arrive(&S.l_bar);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.l_bar);
       if (!warp_wait(&S.l_bar, ne & 1, p.status, ab, false)) break;
       const float lt = l + S.lsum[tid ^ 64];
       const float inv = lt > 0.f ? 1.f / lt : 0.f;
