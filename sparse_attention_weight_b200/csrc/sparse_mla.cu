@@ -93,8 +93,8 @@ constexpr uint32_t kOCol = 256;       // TMEM columns [256,512): O (2 x 128)
 
 struct MlaSmem {
   uint8_t q[kDChunks][kHeads * 128];         // 72 KB  Q of this CTA's heads (K-major SW128)
-  uint8_t s_ring[kSStages][kRows * 128];     // 64 KB  S operand chunks: 128 rows x 64 dims
-  uint8_t v_ring[kVStages][4][kVRows * 128]; // 48 KB  V slices: 4 dim groups x 32 rows (MN-major SW128)
+  uint8_t s_ring[kSStages][kRows * 128];     // 48 KB  S operand chunks: 128 rows x 64 dims
+  uint8_t v_ring[kVStages][4][kVRows * 128]; // 64 KB  V slices: 4 dim groups x 32 rows (MN-major SW128)
   uint8_t p[kBlk / 64][kHeads * 128];        // 32 KB  P: 64 heads x 256 rows (four K chunks of 64 rows)
   float xmax[2][128];
   float lsum[128];
