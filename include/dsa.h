@@ -98,6 +98,7 @@ typedef struct dsa_batch {
 #define DSA_OP_FORWARD 3
 #define DSA_OP_PROJECT 4
 #define DSA_OP_MLA_BACKWARD 5
+#define DSA_OP_FORWARD_HOST 6
 
 /*
  * Bytes of workspace `ws` an operation needs (always >= 256: the status word and
@@ -248,6 +249,41 @@ dsa_status dsa_forward(const dsa_batch *batch, const uint8_t *q_idx, const uint8
                        const float *w, int H_I, const uint16_t *q, const uint16_t *kv, int H, int k,
                        float sm_scale, uint16_t *out, float *lse, void *ws, size_t ws_bytes,
                        void *stream);
+
+/*
+ * dsa_forward for inputs and output held in pinned host memory, with the copies
+ * overlapped with the computation.  The method has no counterpart for this
+ * entry point; it serves callers whose queries arrive from, and whose outputs go
+ * back to, the host.  The queries are processed in chunks of
+ * consecutive rows (each chunk is an independent dsa_forward over the same
+ * cache, so the results are those of dsa_forward on the chunk's queries): the
+ * cache and chunk c+1's queries are copied in on streams[0] while chunk c
+ * computes on streams[1] and chunk c-1's output is copied out on streams[2].
+ *   h_q_idx, h_w, h_q   (pinned host) query-side inputs, layouts as in dsa_forward
+ *   h_k_idx, h_kv       (pinned host) the cache, batch->kv_rows rows of each
+ *   q_idx, w, q, k_idx, kv (device) buffers of the same sizes, overwritten with
+ *                       the copies
+ *   out, lse            (device) as in dsa_forward (lse may be NULL)
+ *   h_out               (pinned host) receives a copy of out
+ *   streams             three streams (copy-in, compute, copy-out; they may be
+ *                       the same stream, which serialises everything)
+ * The call first orders itself after all work already queued on the three
+ * streams that touches these buffers: copies in wait for the compute stream,
+ * the computation waits for the copy-out stream.  When it returns, every copy
+ * and kernel of the call has been queued and the compute stream waits for the
+ * last copy out: once work queued on streams[1] after this call has
+ * completed, h_out holds the output.  The host buffers must stay allocated and
+ * unchanged until then (the copies read and write them asynchronously).
+ * Host pointers must be page-locked (cudaHostAlloc / cudaHostRegister):
+ * pageable memory returns DSA_ERR_UNSUPPORTED.
+ * Workspace: dsa_workspace_size(DSA_OP_FORWARD_HOST, batch, H_I, H, k, 0) (it
+ * covers the largest chunk's forward workspace).  On DSA_ERR_CUDA part of the
+ * work may already be queued.
+ */
+dsa_status dsa_forward_host(const dsa_batch *batch, const uint8_t *h_q_idx, const float *h_w, const uint16_t *h_q,
+                            const uint8_t *h_k_idx, const uint16_t *h_kv, uint8_t *q_idx, float *w, uint16_t *q,
+                            uint8_t *k_idx, uint16_t *kv, int H_I, int H, int k, float sm_scale, uint16_t *out,
+                            float *lse, uint16_t *h_out, void *ws, size_t ws_bytes, void *const streams[3]);
 
 /*
  * Lightning indexer scores for callers that cannot allocate device memory.

@@ -21,12 +21,13 @@ DSA_OK = 0
 STATUS_NAMES = {0: "DSA_OK", 1: "DSA_ERR_INVALID_ARGUMENT", 2: "DSA_ERR_UNSUPPORTED",
                 3: "DSA_ERR_WORKSPACE_TOO_SMALL", 4: "DSA_ERR_CUDA", 5: "DSA_ERR_DEVICE"}
 DEV_BAD_QUERY, DEV_BAD_INDEX, DEV_TIMEOUT = 1, 2, 4
-OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_PROJECT, OP_MLA_BACKWARD = 0, 1, 2, 3, 4, 5
+OP_INDEXER, OP_TOPK, OP_SPARSE_MLA, OP_FORWARD, OP_PROJECT, OP_MLA_BACKWARD, OP_FORWARD_HOST = 0, 1, 2, 3, 4, 5, 6
 
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward",
            "dsa_forward_ws_views", "dsa_read_device_status", "dsa_status_string", "dsa_abi_version",
            "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout", "dsa_launch_count", "dsa_project_append",
-           "dsa_indexer_scores_hist", "dsa_topk_hist", "dsa_topk_uses_hist", "dsa_sparse_mla_backward")
+           "dsa_indexer_scores_hist", "dsa_topk_hist", "dsa_topk_uses_hist", "dsa_sparse_mla_backward",
+           "dsa_forward_host")
 NOALLOC_MAX_Q = 16384
 
 
@@ -72,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_topk_hist.argtypes = [bp, vp, i64, vp, i32, vp, vp, sz, vp]
         L.dsa_topk_uses_hist.argtypes = [bp, i32]
         L.dsa_sparse_mla_backward.argtypes = [bp, vp, vp, vp, i32, i32, f32, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.dsa_forward_host.argtypes = [bp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, f32, vp, vp, vp,
+                                       vp, sz, ctypes.POINTER(vp)]
         L.dsa_topk_uses_hist.restype = i32
         L.dsa_selftest_wait_timeout.argtypes = [vp, sz, ctypes.c_uint32, vp]
         L.dsa_forward_ws_views.argtypes = [bp, i32, i32, i32, vp, ctypes.POINTER(vp), ctypes.POINTER(i64),
@@ -83,7 +86,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_launch_count.restype = ctypes.c_uint64
         for fn in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla", "dsa_forward", "dsa_forward_ws_views",
                    "dsa_read_device_status", "dsa_indexer_scores_noalloc", "dsa_selftest_wait_timeout",
-                   "dsa_project_append", "dsa_indexer_scores_hist", "dsa_topk_hist", "dsa_sparse_mla_backward"):
+                   "dsa_project_append", "dsa_indexer_scores_hist", "dsa_topk_hist", "dsa_sparse_mla_backward",
+                   "dsa_forward_host"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -182,6 +186,20 @@ def dsa_sparse_mla(batch: DeviceBatch, q, kv, idx, k: int, H: int, sm_scale: flo
     _check("dsa_sparse_mla", lib().dsa_sparse_mla(
         ctypes.byref(batch.struct), _ptr(q), _ptr(kv), _ptr(idx), k, H, sm_scale, _ptr(out), _ptr(lse), _ptr(ws),
         ws.numel(), _stream(stream)))
+
+
+def dsa_forward_host(batch: DeviceBatch, host: dict, dev: dict, H_I: int, H: int, k: int, sm_scale: float, out,
+                     lse, h_out, ws, streams=None):
+    """dsa_forward from pinned host tensors `host` (q_idx, w, q, k_idx, kv) through the
+    device buffers `dev` (same names), output copied into the pinned `h_out`;
+    `streams` = (copy-in, compute, copy-out), default: the current stream thrice."""
+    if streams is None:
+        streams = (None, None, None)
+    arr = (ctypes.c_void_p * 3)(*(_stream(s) for s in streams))
+    _check("dsa_forward_host", lib().dsa_forward_host(
+        ctypes.byref(batch.struct), _ptr(host["q_idx"]), _ptr(host["w"]), _ptr(host["q"]), _ptr(host["k_idx"]),
+        _ptr(host["kv"]), _ptr(dev["q_idx"]), _ptr(dev["w"]), _ptr(dev["q"]), _ptr(dev["k_idx"]), _ptr(dev["kv"]),
+        H_I, H, k, sm_scale, _ptr(out), _ptr(lse), _ptr(h_out), _ptr(ws), ws.numel(), arr))
 
 
 def dsa_indexer_scores_hist(batch: DeviceBatch, q_idx, k_idx, w, H_I: int, scores, ld: int, hist, ws, stream=None):

@@ -182,6 +182,64 @@ WsLayout layout(void* ws, int op, const dsa_batch* b, int H, int k, int64_t ld) 
 
 dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
+// dsa_forward_host: about eight query chunks of at least 256 queries (so a chunk
+// fills the sparse-MLA kernel's pairs without split-KV when T is large).
+constexpr int kHostChunks = 8;
+constexpr int kHostMinChunk = 256;
+int host_chunk(int T) {
+  const int c = (T + kHostChunks - 1) / kHostChunks;
+  return c < kHostMinChunk ? kHostMinChunk : c;
+}
+// The queries [q0, q0 + n) of a batch, against the same cache.
+dsa_batch chunk_batch(const dsa_batch* b, int q0, int n) {
+  dsa_batch s = *b;
+  s.num_q = n;
+  s.q_seq = b->q_seq + q0;
+  s.q_pos = b->q_pos + q0;
+  return s;
+}
+// The largest forward workspace of the chunks (a short last chunk may need the
+// split-KV partials that the full-size chunks do not).
+size_t host_ws_bytes(const dsa_batch* b, int H, int k) {
+  const int T = b->num_q, c = host_chunk(T);
+  size_t m = kWsHeader;
+  for (int q0 = 0; q0 < T; q0 += c) {
+    const dsa_batch s = chunk_batch(b, q0, T - q0 < c ? T - q0 : c);
+    const size_t n = layout(nullptr, DSA_OP_FORWARD, &s, H, k, default_ld(b)).bytes;
+    if (n > m) m = n;
+  }
+  return m;
+}
+bool pinned_host(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+// Events of one call, destroyed on every return path (a recorded event is
+// released by the driver once it completes).
+struct EventSet {
+  cudaEvent_t e[4 + 2 * (kHostChunks + 1)];
+  int n = 0;
+  cudaEvent_t make() {
+    if (n == static_cast<int>(sizeof(e) / sizeof(e[0]))) return nullptr;
+    cudaEvent_t x = nullptr;
+    if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    e[n++] = x;
+    return x;
+  }
+  ~EventSet() {
+    for (int i = 0; i < n; ++i) cudaEventDestroy(e[i]);
+  }
+};
+// `to` waits for the work queued so far on `from`.
+bool order_after(EventSet& E, cudaStream_t from, cudaStream_t to) {
+  cudaEvent_t x = E.make();
+  return x && cudaEventRecord(x, from) == cudaSuccess && cudaStreamWaitEvent(to, x, 0) == cudaSuccess;
+}
+
 dsa_status run_indexer(const dsa_batch* b, const uint8_t* q_idx, const uint8_t* k_idx, const float* w, int H_I,
                        float* scores, int64_t ld, const WsLayout& L, cudaStream_t st, uint32_t* hist = nullptr) {
   if (b->num_q == 0) return DSA_OK;
@@ -288,6 +346,7 @@ size_t dsa_workspace_size(int op, const dsa_batch* batch, int H_I, int H, int k,
   if (!batch_ok(batch)) return 0;
   if (op == DSA_OP_PROJECT) return hi_ok(H_I) && h_ok(H) ? proj_layout(nullptr, batch, H_I, H).bytes : 0;
   if (op == DSA_OP_MLA_BACKWARD) return kWsHeader;
+  if (op == DSA_OP_FORWARD_HOST) return hi_ok(H_I) && h_ok(H) && k_ok(k) ? host_ws_bytes(batch, H, k) : 0;
   if (op < DSA_OP_INDEXER || op > DSA_OP_FORWARD) return 0;
   if ((op == DSA_OP_SPARSE_MLA || op == DSA_OP_FORWARD) && (!h_ok(H) || !k_ok(k))) return 0;
   if (op == DSA_OP_FORWARD && !k_ok(k)) return 0;
@@ -483,6 +542,66 @@ dsa_status dsa_project_append(const dsa_batch* batch, const uint16_t* hidden, co
   const cudaError_t e = launch_project(p, hidden, w_all, d_model, L.gemm_ws, project_gemm_workspace_bytes(), st,
                                        &gemm_failed);
   return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status dsa_forward_host(const dsa_batch* batch, const uint8_t* h_q_idx, const float* h_w, const uint16_t* h_q,
+                            const uint8_t* h_k_idx, const uint16_t* h_kv, uint8_t* q_idx, float* w, uint16_t* q,
+                            uint8_t* k_idx, uint16_t* kv, int H_I, int H, int k, float sm_scale, uint16_t* out,
+                            float* lse, uint16_t* h_out, void* ws, size_t ws_bytes, void* const streams[3]) {
+  if (!batch_ok(batch) || !ws || !streams) return DSA_ERR_INVALID_ARGUMENT;
+  const int T = batch->num_q;
+  if (T > 0 && (!h_q_idx || !h_w || !h_q || !h_k_idx || !h_kv || !q_idx || !w || !q || !k_idx || !kv || !out ||
+                !h_out))
+    return DSA_ERR_INVALID_ARGUMENT;
+  if (!hi_ok(H_I) || !h_ok(H) || !k_ok(k) || !paging_ok(batch)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(q) || !aligned16(kv) ||
+      !aligned16(out) || !aligned16(ws))
+    return DSA_ERR_UNSUPPORTED;
+  if (ws_bytes < host_ws_bytes(batch, H, k)) return DSA_ERR_WORKSPACE_TOO_SMALL;
+  if (T > 0 && (!pinned_host(h_q_idx) || !pinned_host(h_w) || !pinned_host(h_q) || !pinned_host(h_k_idx) ||
+                !pinned_host(h_kv) || !pinned_host(h_out)))
+    return DSA_ERR_UNSUPPORTED;
+  cudaStream_t s_in = static_cast<cudaStream_t>(streams[0]);
+  cudaStream_t s_cp = static_cast<cudaStream_t>(streams[1]);
+  cudaStream_t s_out = static_cast<cudaStream_t>(streams[2]);
+  EventSet E;
+  // after the earlier copies out of `out`, then the earlier readers of the inputs
+  if (!order_after(E, s_out, s_cp) || !order_after(E, s_cp, s_in)) return DSA_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, sizeof(uint32_t), s_cp) != cudaSuccess) return DSA_ERR_CUDA;
+  if (T == 0) return DSA_OK;
+  const size_t rows = static_cast<size_t>(batch->kv_rows);
+  if (cudaMemcpyAsync(k_idx, h_k_idx, rows * DSA_D_INDEX, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+      cudaMemcpyAsync(kv, h_kv, rows * DSA_D_QK * 2, cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+      !order_after(E, s_in, s_cp))
+    return DSA_ERR_CUDA;
+  const int64_t ld = default_ld(batch);
+  const int c = host_chunk(T);
+  for (int q0 = 0; q0 < T; q0 += c) {
+    const int n = T - q0 < c ? T - q0 : c;
+    const size_t o_qi = static_cast<size_t>(q0) * H_I * DSA_D_INDEX, o_w = static_cast<size_t>(q0) * H_I;
+    const size_t o_q = static_cast<size_t>(q0) * H * DSA_D_QK, o_o = static_cast<size_t>(q0) * H * DSA_D_V;
+    if (cudaMemcpyAsync(q_idx + o_qi, h_q_idx + o_qi, static_cast<size_t>(n) * H_I * DSA_D_INDEX,
+                        cudaMemcpyHostToDevice, s_in) != cudaSuccess ||
+        cudaMemcpyAsync(w + o_w, h_w + o_w, static_cast<size_t>(n) * H_I * sizeof(float), cudaMemcpyHostToDevice,
+                        s_in) != cudaSuccess ||
+        cudaMemcpyAsync(q + o_q, h_q + o_q, static_cast<size_t>(n) * H * DSA_D_QK * 2, cudaMemcpyHostToDevice,
+                        s_in) != cudaSuccess ||
+        !order_after(E, s_in, s_cp))
+      return DSA_ERR_CUDA;
+    const dsa_batch sub = chunk_batch(batch, q0, n);
+    const WsLayout L = layout(ws, DSA_OP_FORWARD, &sub, H, k, ld);
+    dsa_status st = run_indexer(&sub, q_idx + o_qi, k_idx, w + o_w, H_I, L.scores, ld, L, s_cp);
+    if (st == DSA_OK) st = run_topk(&sub, L.scores, ld, k, L.idx, L, s_cp);
+    if (st == DSA_OK)
+      st = run_mla(&sub, q + o_q, kv, L.idx, k, H, sm_scale, out + o_o, lse ? lse + static_cast<size_t>(q0) * H : nullptr,
+                   L, s_cp);
+    if (st != DSA_OK) return st;
+    if (!order_after(E, s_cp, s_out) ||
+        cudaMemcpyAsync(h_out + o_o, out + o_o, static_cast<size_t>(n) * H * DSA_D_V * 2, cudaMemcpyDeviceToHost,
+                        s_out) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  return order_after(E, s_out, s_cp) ? DSA_OK : DSA_ERR_CUDA;
 }
 
 dsa_status dsa_forward_ws_views(const dsa_batch* batch, int H_I, int H, int k, void* ws, float** scores, int64_t* ld,

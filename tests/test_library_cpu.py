@@ -148,6 +148,32 @@ def test_histogram_fusion_host_checks(lib):
     assert lib.dsa_topk_uses_hist(None, 2048) == 0
 
 
+def test_forward_host_host_checks(lib):
+    """dsa_forward_host: the workspace covers the largest query chunk (a short last
+    chunk may take split-KV partials that a full-size one does not), and bad
+    arguments are refused before any copy is queued."""
+    ws, p, big = 0x50000, 0x60000, 1 << 40
+    for T in (16, 700, 5000):
+        b = _fake_batch(T=T)
+        host = lib.dsa_workspace_size(B.OP_FORWARD_HOST, ctypes.byref(b), 64, 128, 2048, 0)
+        fwd = lib.dsa_workspace_size(B.OP_FORWARD, ctypes.byref(b), 64, 128, 2048, 0)
+        assert host > 0 and fwd > 0
+        # chunks of max(256, ceil(T/8)) queries: at most one chunk's scores and indices
+        chunk = max(256, -(-T // 8))
+        assert host >= min(T, chunk) * (3000 * 4 + 2048 * 4)
+        assert host <= fwd + 64 * 2 * 128 * 512 * 4 + (1 << 20)
+    assert lib.dsa_workspace_size(B.OP_FORWARD_HOST, ctypes.byref(_fake_batch()), 64, 12, 2048, 0) == 0
+    b = _fake_batch()
+    streams = (ctypes.c_void_p * 3)(None, None, None)
+    call = lambda **kw: lib.dsa_forward_host(
+        ctypes.byref(b), kw.get("hq", p), p, p, p, p, p, p, p, p, p, kw.get("hi", 64), 128, 2048, 0.1, p, None,
+        kw.get("hout", p), ws, kw.get("ws_bytes", big), kw.get("streams", streams))
+    assert call(streams=None) == 1                      # no stream array
+    assert call(hq=0) == 1 and call(hout=0) == 1         # null host buffers
+    assert call(hi=10) == 2
+    assert call(ws_bytes=1024) == 3
+
+
 def test_read_device_status_rejects_null(lib):
     flags = ctypes.c_uint32()
     assert lib.dsa_read_device_status(None, ctypes.byref(flags), None) == 1
