@@ -59,7 +59,7 @@ D_QK, D_V, D_INDEX = 576, 512, 128
 # `bench.py --seq-len 2304 --steps 1 --warmup 1 --no-e2e --no-cpu-baseline`,
 # divided by its 2304 queries (the traffic is the queries in and the outputs out;
 # the gathered cache rows hit L2).  None while no capture describes the kernel.
-MLA_TRAFFIC_BYTES_PER_QUERY = (361.408e6 + 259.017216e6) / 2304
+MLA_TRAFFIC_BYTES_PER_QUERY = (361.410816e6 + 257.011456e6) / 2304
 # Workloads run with a paged cache, and their page size (rows).
 PAGED = {"decode_b1_128k": 64}
 
