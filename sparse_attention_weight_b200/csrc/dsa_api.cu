@@ -182,9 +182,9 @@ WsLayout layout(void* ws, int op, const dsa_batch* b, int H, int k, int64_t ld) 
 
 dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
-// dsa_forward_host: about eight query chunks of at least 256 queries (so a chunk
+// dsa_forward_host: about sixteen query chunks of at least 256 queries (so a chunk
 // fills the sparse-MLA kernel's pairs without split-KV when T is large).
-constexpr int kHostChunks = 8;
+constexpr int kHostChunks = 16;
 constexpr int kHostMinChunk = 256;
 int host_chunk(int T) {
   const int c = (T + kHostChunks - 1) / kHostChunks;

@@ -159,7 +159,7 @@ def test_forward_host_host_checks(lib):
         fwd = lib.dsa_workspace_size(B.OP_FORWARD, ctypes.byref(b), 64, 128, 2048, 0)
         assert host > 0 and fwd > 0
         # chunks of max(256, ceil(T/8)) queries: at most one chunk's scores and indices
-        chunk = max(256, -(-T // 8))
+        chunk = max(256, -(-T // 16))
         assert host >= min(T, chunk) * (3000 * 4 + 2048 * 4)
         assert host <= fwd + 64 * 2 * 128 * 512 * 4 + (1 << 20)
     assert lib.dsa_workspace_size(B.OP_FORWARD_HOST, ctypes.byref(_fake_batch()), 64, 12, 2048, 0) == 0
