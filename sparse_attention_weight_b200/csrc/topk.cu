@@ -8,14 +8,17 @@
 //
 // Design.  One CTA per query row.  Scores map to order-preserving 32-bit keys;
 // the k-th largest key is found exactly by three histogram passes over 11, 11
-// and 10 key bits (2048-bin shared-memory histograms, warp-aggregated with
-// match.any so hot bins take one atomic per warp), then one output pass emits,
+// and 10 key bits (2048-bin shared-memory histograms; a warp whose keys share
+// one bin makes one atomic, found with ballots), then one output pass emits,
 // in index order, every key above the threshold and the first `need` keys equal
 // to it.  The output pass needs a single block scan per 2048 elements: with
 // gt/eq counts before an element, its slot is gt_before + min(eq_before, need).
 // Rows up to the shared-memory cache size are read from HBM once; longer rows
 // are re-read from L2 by each pass.  Loads are float4 (16 B per thread,
-// 512 B per warp, coalesced).
+// 512 B per warp, coalesced).  A cached row of at least 5k keys whose keys at
+// or above the first pass's bin fit a list (and are at most a quarter of the
+// row) is compacted, in index order, into that list of positions, and the two
+// later passes and the output run over the list instead of the whole row.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -29,6 +32,13 @@ constexpr int kStep = kThreads * kPer;   // elements per block step
 constexpr int kCacheMax = 32768;         // keys cached in shared memory at most (128 KB)
 constexpr int kClusterMinLen = 8192;     // rows at least this long may share a cluster of CTAs
 constexpr int kClusterSegMax = 20480;    // keys cached per CTA of a cluster (80 KB: two CTAs per SM)
+// Cached rows: positions of the keys at or above the pass-1 threshold bin, in
+// index order (about k plus one bin), so that the later passes and the output
+// run over this list instead of the whole cached row.  The host sizes the list
+// within the shared memory left over at the kernel's occupancy (at most this
+// many entries); a row segment whose list would be longer than that, or than a
+// quarter of the segment, takes the passes over the cache.
+constexpr int kRowListMax = 3072;
 
 struct Ctx {
   const float* row;
@@ -170,12 +180,111 @@ __device__ __forceinline__ int row_length(const TopkParams& p, int t, int32_t* o
   return n;
 }
 
+// Ordered compaction of a cached row segment: the positions of its keys whose
+// top 11 bits are >= b1, in index order, into `list`; returns their number.
+// One block scan per 2048 keys.
+__device__ int compact_at_or_above(const uint32_t* cache, int m, uint32_t b1, int32_t* list, uint32_t* scratch) {
+  int out_base = 0;
+  for (int base = 0; base < m; base += kStep) {
+    const int i = base + threadIdx.x * kPer;
+    const uint4 v = *reinterpret_cast<const uint4*>(cache + i);   // the cache is whole steps long
+    const uint32_t kk[kPer] = {v.x, v.y, v.z, v.w};
+    uint32_t cnt = 0;
+    bool f[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      f[u] = (i + u) < m && (kk[u] >> 21) >= b1;
+      cnt += f[u] ? 1u : 0u;
+    }
+    uint32_t total;
+    const uint32_t incl = block_scan(cnt, scratch, &total);
+    int pos = out_base + static_cast<int>(incl - cnt);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u)
+      if (f[u]) list[pos++] = i + u;
+    out_base += static_cast<int>(total);
+  }
+  return out_base;
+}
+
+// hist_pass over the listed keys of a cached row.
+__device__ void hist_listed(const uint32_t* cache, const int32_t* list, int m, uint32_t* hist, int shift, int bits,
+                            int fshift, uint32_t prefix) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t mask = (1u << bits) - 1u;
+  for (int base = 0; base < m; base += kThreads) {
+    const int i = base + threadIdx.x;
+    const uint32_t key = i < m ? cache[list[i]] : 0u;
+    hist_add(hist, (key >> shift) & mask, i < m && (key >> fshift) == prefix, lane);
+  }
+}
+
+// Counts of listed keys above / equal to tau.
+__device__ void count_listed(const uint32_t* cache, const int32_t* list, int m, uint32_t tau, uint32_t& cgt,
+                             uint32_t& ceq) {
+  cgt = 0;
+  ceq = 0;
+  for (int i = threadIdx.x; i < m; i += kThreads) {
+    const uint32_t key = cache[list[i]];
+    cgt += key > tau ? 1u : 0u;
+    ceq += key == tau ? 1u : 0u;
+  }
+}
+
+// Output pass over the listed keys (index order, four per thread per step):
+// every key above tau and the first `need` keys equal to it, at slots after
+// gt_base / eq_base earlier ones; `lo` is the global index of the cached
+// segment's first key.
+__device__ void output_listed(const uint32_t* cache, const int32_t* list, int m, uint32_t tau, uint32_t need, int k,
+                              int lo, uint32_t gt_base, uint32_t eq_base, int32_t* out, uint32_t* scratch) {
+  for (int base = 0; base < m; base += kStep) {
+    const int i = base + threadIdx.x * kPer;
+    int pos[kPer];
+    uint32_t kk[kPer];
+    bool valid[kPer];
+    uint32_t cgt = 0, ceq = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      valid[u] = i + u < m;
+      pos[u] = valid[u] ? list[i + u] : 0;
+      kk[u] = valid[u] ? cache[pos[u]] : 0u;
+      cgt += (valid[u] && kk[u] > tau) ? 1u : 0u;
+      ceq += (valid[u] && kk[u] == tau) ? 1u : 0u;
+    }
+    const uint32_t packed = cgt | (ceq << 16);
+    uint32_t total;
+    const uint32_t excl = block_scan(packed, scratch, &total) - packed;
+    uint32_t gt_before = gt_base + (excl & 0xffffu);
+    uint32_t eq_before = eq_base + (excl >> 16);
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (!valid[u]) continue;
+      if (kk[u] > tau) {
+        const uint32_t slot = gt_before + min(eq_before, need);
+        if (slot < static_cast<uint32_t>(k)) out[slot] = lo + pos[u];
+        ++gt_before;
+      } else if (kk[u] == tau) {
+        const uint32_t slot = gt_before + eq_before;
+        if (eq_before < need && slot < static_cast<uint32_t>(k)) out[slot] = lo + pos[u];
+        ++eq_before;
+      }
+    }
+    gt_base += total & 0xffffu;
+    eq_base += total >> 16;
+  }
+}
+
+// A list pays when it holds at most a quarter of the segment's keys.
+__device__ __forceinline__ bool use_list(uint32_t at_or_above, int list_cap, int m) {
+  return at_or_above <= static_cast<uint32_t>(list_cap) && 4u * at_or_above <= static_cast<uint32_t>(m);
+}
+
 // Exact top-k of row c (n > k) by three histogram passes (11, 11, 10 key bits)
 // and one output pass over the row: from the shared-memory cache when c.cache
 // is set (the first pass fills it), from L2 otherwise.  An uncached row whose
 // first histogram the indexer already emitted (hist_in) skips the first pass.
 __device__ void select_streaming(const Ctx& c, int k, int32_t* out, uint32_t* hist, uint32_t* scratch,
-                                 uint32_t* sel, const uint32_t* hist_in) {
+                                 uint32_t* sel, const uint32_t* hist_in, int32_t* list, int list_cap) {
   const bool cached = c.cache != nullptr;
   const int n = c.n;
   // pass 1: bits 31..21
@@ -190,7 +299,30 @@ __device__ void select_streaming(const Ctx& c, int k, int32_t* out, uint32_t* hi
   }
   find_bin(hist, 2048, static_cast<uint32_t>(k), scratch, &sel[0], &sel[1]);
   const uint32_t b1 = sel[0], r1 = sel[1];
+  // keys at or above bin b1: the k - r1 above it and the bin's own
+  const uint32_t at_or_above = static_cast<uint32_t>(k) - r1 + hist[b1];
   __syncthreads();
+
+  if (cached && list && use_list(at_or_above, list_cap, n)) {
+    // the remaining passes and the output over the listed keys only
+    const int m = compact_at_or_above(c.cache, n, b1, list, scratch);
+    for (int b = threadIdx.x; b < 2048; b += kThreads) hist[b] = 0;
+    __syncthreads();
+    hist_listed(c.cache, list, m, hist, 10, 11, 21, b1);
+    __syncthreads();
+    find_bin(hist, 2048, r1, scratch, &sel[0], &sel[1]);
+    const uint32_t pre2 = (b1 << 11) | sel[0], r2 = sel[1];
+    __syncthreads();
+    for (int b = threadIdx.x; b < 1024; b += kThreads) hist[b] = 0;
+    __syncthreads();
+    hist_listed(c.cache, list, m, hist, 0, 10, 10, pre2);
+    __syncthreads();
+    find_bin(hist, 1024, r2, scratch, &sel[0], &sel[1]);
+    const uint32_t tau = (pre2 << 10) | sel[0], need = sel[1];
+    __syncthreads();
+    output_listed(c.cache, list, m, tau, need, k, 0, 0u, 0u, out, scratch);
+    return;
+  }
 
   // pass 2: bits 20..10 among keys with the pass-1 prefix
   for (int b = threadIdx.x; b < 2048; b += kThreads) hist[b] = 0;
@@ -249,18 +381,20 @@ __device__ void select_streaming(const Ctx& c, int k, int32_t* out, uint32_t* hi
   }
 }
 
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p, int cache_elems) {
+__global__ void __launch_bounds__(kThreads) topk_kernel(TopkParams p, int cache_elems, int list_cap) {
   extern __shared__ __align__(16) uint32_t tk_smem[];
   uint32_t* hist = tk_smem;                 // 2048
   uint32_t* scratch = hist + 2048;          // 32
   uint32_t* sel = scratch + 32;             // [0] bin, [1] remaining
   uint32_t* cache = sel + 32;               // cache_elems (16-byte aligned: offset 2112 words)
+  int32_t* list = list_cap > 0 ? reinterpret_cast<int32_t*>(cache + cache_elems) : nullptr;   // list_cap
   const int t = blockIdx.x;
   int32_t* out = p.idx + static_cast<int64_t>(t) * p.k;
   const int n = row_length(p, t, out);
   if (n <= 0) return;
   const Ctx c{p.scores + static_cast<int64_t>(t) * p.ld, n <= cache_elems ? cache : nullptr, n};
-  select_streaming(c, p.k, out, hist, scratch, sel, p.hist ? p.hist + static_cast<int64_t>(t) * 2048 : nullptr);
+  select_streaming(c, p.k, out, hist, scratch, sel, p.hist ? p.hist + static_cast<int64_t>(t) * 2048 : nullptr,
+                   list, list_cap);
 }
 
 // ---------------------------------------------------------------- long rows
@@ -313,7 +447,7 @@ __global__ void __launch_bounds__(kThreads) topk_long_kernel(TopkParams p) {
   const uint32_t m_total = (static_cast<uint32_t>(k) - r1) + hist[b1];   // keys at or above bin b1
   __syncthreads();
   if (m_total > static_cast<uint32_t>(kListCap)) {    // block-uniform: fall back to streaming
-    select_streaming(c, k, out, hist, scratch, sel, nullptr);
+    select_streaming(c, k, out, hist, scratch, sel, nullptr, nullptr, 0);
     return;
   }
 
@@ -458,10 +592,11 @@ __device__ __forceinline__ void cl_push(const ClusterShared& S, uint32_t* dst, i
   }
 }
 
-__global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, int seg_cap) {
+__global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, int seg_cap, int list_cap) {
   extern __shared__ __align__(16) uint32_t tk_smem[];
   ClusterShared& S = *reinterpret_cast<ClusterShared*>(tk_smem);
   uint32_t* cache = tk_smem + (sizeof(ClusterShared) + 15) / 16 * 4;   // seg_cap keys
+  int32_t* list = reinterpret_cast<int32_t*>(cache + seg_cap);          // list_cap positions
   const uint32_t C = cl_size(), r = cl_rank();
   const int t = blockIdx.x / static_cast<int>(C);
   const int k = p.k;
@@ -542,6 +677,19 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, in
   const uint32_t b1 = S.sel[0], r1 = S.sel[1];
   __syncthreads();
 
+  // This segment's keys at or above bin b1 (from its own pass-1 histogram): when
+  // they fit the list, the later passes and the output run over their positions
+  // only.  Each CTA decides for itself; the cluster steps below are the same.
+  bool listed = false;
+  if (!have_hist && list_cap > 0) {                        // uniform over the grid
+    uint32_t mine = 0;
+    for (int b = threadIdx.x; b < 2048; b += kThreads) mine += b >= static_cast<int>(b1) ? S.local[b] : 0u;
+    uint32_t at_or_above;
+    block_scan(mine, S.scratch, &at_or_above);
+    listed = use_list(at_or_above, list_cap, m);
+  }
+  const int ml = listed ? compact_at_or_above(cache, m, b1, list, S.scratch) : 0;
+
   // pass 2: bits 20..10 of the keys with the pass-1 prefix (global[1] was cleared at the start)
   for (int b = threadIdx.x; b < 2048; b += kThreads) {
     S.local[b] = 0;
@@ -549,7 +697,8 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, in
   }
   __syncthreads();
   const Ctx cc{nullptr, cache, m};
-  hist_pass(cc, true, false, S.local, 10, 11, 21, b1);
+  if (listed) hist_listed(cache, list, ml, S.local, 10, 11, 21, b1);
+  else hist_pass(cc, true, false, S.local, 10, 11, 21, b1);
   __syncthreads();
   cl_push(S, S.global[1], 2048, C);
   cl_sync();
@@ -561,7 +710,8 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, in
   const uint32_t pre2 = (b1 << 11) | b2;
   for (int b = threadIdx.x; b < 2048; b += kThreads) S.local[b] = 0;
   __syncthreads();
-  hist_pass(cc, true, false, S.local, 0, 10, 10, pre2);
+  if (listed) hist_listed(cache, list, ml, S.local, 0, 10, 10, pre2);
+  else hist_pass(cc, true, false, S.local, 0, 10, 10, pre2);
   __syncthreads();
   cl_push(S, S.global[0], 1024, C);
   cl_sync();
@@ -573,10 +723,14 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, in
   // counts above / equal to tau of every segment -> offsets of this segment's output
   {
     uint32_t cgt = 0, ceq = 0;
-    for (int i = threadIdx.x; i < m; i += kThreads) {
-      const uint32_t key = cache[i];
-      cgt += key > tau ? 1u : 0u;
-      ceq += key == tau ? 1u : 0u;
+    if (listed) {
+      count_listed(cache, list, ml, tau, cgt, ceq);
+    } else {
+      for (int i = threadIdx.x; i < m; i += kThreads) {
+        const uint32_t key = cache[i];
+        cgt += key > tau ? 1u : 0u;
+        ceq += key == tau ? 1u : 0u;
+      }
     }
     uint32_t tgt, teq;
     block_scan(cgt, S.scratch, &tgt);
@@ -589,6 +743,10 @@ __global__ void __launch_bounds__(kThreads) topk_cluster_kernel(TopkParams p, in
   cl_sync();                                               // last access to another CTA's memory
   uint32_t gt_base = 0, eq_base = 0;
   for (uint32_t c = 0; c < r; ++c) { gt_base += S.cnt_gt[c]; eq_base += S.cnt_eq[c]; }
+  if (listed) {
+    output_listed(cache, list, ml, tau, need, k, lo, gt_base, eq_base, out, S.scratch);
+    return;
+  }
 
   // output pass over the cached segment, index order (global index = lo + i)
   for (int base = 0; base < m; base += kStep) {
@@ -655,6 +813,29 @@ bool topk_uses_hist(int max_kv_len, int T, int sms) {
   return plan >= 2 || plan == -1;
 }
 
+// A list is allocated only for rows of at least 5k keys (it must stay within a
+// quarter of them) and, in a cluster, only when it can hold a segment's share of
+// about 1.5k keys.
+// Entries of a row list that fit in the shared memory a CTA of `base` bytes
+// leaves over at its occupancy without one (at most four 512-thread CTAs per
+// SM); 0 when fewer than 512 fit.
+int list_cap_for(size_t base, int dev) {
+  int per_sm = 0, reserved = 0, per_block = 0;
+  if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&per_block, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+    return 0;
+  const size_t slot = base + static_cast<size_t>(reserved);
+  size_t ctas = static_cast<size_t>(per_sm) / slot;
+  if (ctas == 0) return 0;
+  if (ctas > 4) ctas = 4;
+  size_t room = static_cast<size_t>(per_sm) / ctas - slot;
+  if (base + room > static_cast<size_t>(per_block)) room = base < static_cast<size_t>(per_block) ? per_block - base : 0;
+  size_t cap = room / sizeof(int32_t) / 4 * 4;
+  if (cap > static_cast<size_t>(kRowListMax)) cap = kRowListMax;
+  return cap >= 512 ? static_cast<int>(cap) : 0;
+}
+
 cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   int cache_elems = ((p.max_kv_len + kStep - 1) / kStep) * kStep;
@@ -676,7 +857,11 @@ cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
     const int C = c_fit > c_par ? c_fit : c_par;
     if (C >= 2 && C <= 8) {
       const int seg_cap = seg_of(C);
-      const size_t smem = (sizeof(ClusterShared) + 15) / 16 * 16 + static_cast<size_t>(seg_cap) * sizeof(uint32_t);
+      const size_t base = (sizeof(ClusterShared) + 15) / 16 * 16 + static_cast<size_t>(seg_cap) * sizeof(uint32_t);
+      // a segment's list holds about (k + one bin) / C keys
+      int list_cap = p.max_kv_len >= 5 * p.k ? list_cap_for(base, dev) : 0;
+      if (list_cap < (3 * p.k / 2 + C - 1) / C) list_cap = 0;
+      const size_t smem = base + static_cast<size_t>(list_cap) * sizeof(int32_t);
       cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
       if (e != cudaSuccess) return e;
@@ -692,7 +877,7 @@ cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
       attr[0].val.clusterDim.z = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, p, seg_cap);
+      e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel, p, seg_cap, list_cap);
       if (e == cudaSuccess) count_launches(1);
       return e;
     }
@@ -712,11 +897,13 @@ cudaError_t launch_topk(const TopkParams& p, int T, cudaStream_t stream) {
     return e;
   }
   if (cache_elems > kCacheMax) cache_elems = 0;       // long rows stream from L2
-  const size_t smem = (2048 + 64) * sizeof(uint32_t) + static_cast<size_t>(cache_elems) * sizeof(uint32_t);
+  const size_t base = (2048 + 64) * sizeof(uint32_t) + static_cast<size_t>(cache_elems) * sizeof(uint32_t);
+  const int list_cap = cache_elems > 0 && p.max_kv_len >= 5 * p.k ? list_cap_for(base, dev) : 0;
+  const size_t smem = base + static_cast<size_t>(list_cap) * sizeof(int32_t);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  topk_kernel<<<T, kThreads, smem, stream>>>(p, cache_elems);
+  topk_kernel<<<T, kThreads, smem, stream>>>(p, cache_elems, list_cap);
   e = cudaGetLastError();
   if (e == cudaSuccess) count_launches(1);
   return e;
