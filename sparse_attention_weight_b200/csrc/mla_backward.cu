@@ -9,15 +9,21 @@
 //   dQ = s sum_i dZ_i kv_i,   dKV[r_i] += s dZ_i q + p_i [dO, 0]
 // with o and lse the forward's output and log-sum-exp.
 //
-// Design (a first, CUDA-core path).  One CTA per (query, chunk of HC heads):
-// the chunk's queries and output gradients stay in shared memory as fp32, the
-// selected rows stream through in tiles of 16 (gathered by index, converted to
-// fp32); per tile the CTA forms z, p, dZ for the chunk's heads, adds into dQ
-// (registers) and forms each row's dKV contribution summed over the chunk's
-// heads, which it adds to the fp32 gradient cache with vector atomics (a row
-// selected by several queries collects all their contributions).  Rows are
-// padded to an odd stride in shared memory so that threads reading different
-// rows at the same column hit different banks.
+// Design (CUDA cores, fp32).  One CTA (256 threads) per (query, chunk of HC =
+// 32/16/8 heads): the chunk's queries and output gradients stay in shared memory
+// as fp32, the selected rows stream through in tiles of 32 (gathered by index,
+// converted to fp32); a tile without a usable entry is skipped.  Per tile, three
+// register-tiled products:
+//   1. z and dO.v for every (head, row): each thread a 4-head x 4-row tile over a
+//      1/KS slice of the 576 (512) dims, float4 loads, the KS slices summed by
+//      shuffles; then p and dZ, one row per slice lane.
+//   2. dQ += dZ . rows: each thread HC/8 heads x 18 dims, accumulated in
+//      registers over all tiles (written once, no atomics).
+//   3. each row's d_kv contribution summed over the chunk's heads: each thread 4
+//      rows x 18 dims, added to the fp32 gradient cache with float2 atomics (a
+//      row selected by several queries collects all their contributions).
+// Row strides in shared memory are padded by 4 floats (16-byte aligned rows
+// whose banks shift by 4 from one row to the next).
 #include <cuda_bf16.h>
 
 #include "dsa_common.cuh"
@@ -28,9 +34,10 @@ namespace dsa {
 namespace {
 
 constexpr int kBwdThreads = 256;
-constexpr int kRT = 16;                  // selected rows per tile
-constexpr int kQS = DSA_D_QK + 1;        // padded fp32 stride of a 576-wide row
-constexpr int kOS = DSA_D_V + 1;         // padded fp32 stride of a 512-wide row
+constexpr int kRT = 32;                  // selected rows per tile
+constexpr int kQS = DSA_D_QK + 4;        // padded fp32 stride of a 576-wide row
+constexpr int kOS = DSA_D_V + 4;         // padded fp32 stride of a 512-wide row
+constexpr int kDPer = DSA_D_QK / 32;     // 18 dims per lane in products 2 and 3 (float2 pairs lane*2 + 64j)
 
 template <int HC>
 struct BwdSmem {
@@ -53,6 +60,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mla_backward_kernel(MlaBwdPara
   const int t = blockIdx.x;
   const int h0 = blockIdx.y * HC;
   const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int H = p.H;
   // sequence of the query
   const int seq = p.q_seq[t];
@@ -90,22 +98,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mla_backward_kernel(MlaBwdPara
   }
   __syncthreads();
 
-  // dQ accumulators: thread = (head hq, 576 / (256 / HC) consecutive dims)
-  constexpr int QTPH = kBwdThreads / HC;           // threads per head for dQ
-  constexpr int QPER = DSA_D_QK / QTPH;            // dims per thread
-  const int hq = tid / QTPH, dq0 = (tid % QTPH) * QPER;
-  float dq[QPER];
+  // product 1 mapping: tile (hb, rb) of 4 heads x 4 rows, KS lanes per tile
+  constexpr int KS = 128 / HC;                     // 4, 8, 16
+  const int tile = tid / KS, ks = tid % KS;
+  const int hb = tile / (kRT / 4), rb = tile % (kRT / 4);
+  // product 2 mapping: heads warp*HPW .. +HPW-1, dims lane*2 + 64j
+  constexpr int HPW = HC / 8;                      // 4, 2, 1
+  float dq[HPW][kDPer];
 #pragma unroll
-  for (int j = 0; j < QPER; ++j) dq[j] = 0.f;
-  // dKV contributions: thread = (tile row rk, 36 consecutive dims)
-  constexpr int KTPR = kBwdThreads / kRT;          // 16 threads per row
-  constexpr int KPER = DSA_D_QK / KTPR;            // 36 dims per thread
-  const int rk = tid / KTPR, dk0 = (tid % KTPR) * KPER;
+  for (int a = 0; a < HPW; ++a)
+#pragma unroll
+    for (int j = 0; j < kDPer; ++j) dq[a][j] = 0.f;
   const float scale = p.sm_scale;
 
   const int32_t* idx_row = p.idx + static_cast<int64_t>(t) * p.k;
   for (int e0 = 0; rows_ok && e0 < p.k; e0 += kRT) {
     // cache rows of the tile's entries
+    bool any = false;
     if (tid < kRT) {
       const int e = e0 + tid;
       const int v = e < p.k ? idx_row[e] : -1;
@@ -124,75 +133,160 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mla_backward_kernel(MlaBwdPara
         }
       }
       S.row_of[tid] = r;
+      any = r >= 0;
     }
-    __syncthreads();
+    if (!__syncthreads_or(any)) continue;          // no usable entry in this tile
     // gather the rows (8 bf16 per 16-byte load), zeros for unused entries
     for (int i = tid; i < kRT * (DSA_D_QK / 8); i += kBwdThreads) {
       const int r = i / (DSA_D_QK / 8), c8 = i - r * (DSA_D_QK / 8);
       const int64_t row = S.row_of[r];
       uint4 v = make_uint4(0u, 0u, 0u, 0u);
       if (row >= 0) v = __ldg(reinterpret_cast<const uint4*>(p.kv + row * DSA_D_QK) + c8);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      float* dst = &S.rows[r][c8 * 8];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        dst[2 * u] = __uint_as_float(w[u] << 16);
-        dst[2 * u + 1] = __uint_as_float(w[u] & 0xffff0000u);
-      }
+      float4* dst = reinterpret_cast<float4*>(&S.rows[r][c8 * 8]);
+      dst[0] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+      dst[1] = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u),
+                           __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
     }
     __syncthreads();
-    // z, p, dZ for every (head, entry) pair of the tile
-    for (int pr = tid; pr < HC * kRT; pr += kBwdThreads) {
-      const int h = pr / kRT, r = pr - h * kRT;
-      float z = 0.f, dp = 0.f;
-      for (int d = 0; d < DSA_D_V; ++d) {
-        const float kvd = S.rows[r][d];
-        z = fmaf(S.q[h][d], kvd, z);
-        dp = fmaf(S.dout[h][d], kvd, dp);
-      }
-      for (int d = DSA_D_V; d < DSA_D_QK; ++d) z = fmaf(S.q[h][d], S.rows[r][d], z);
-      const bool used = S.row_of[r] >= 0 && S.lse[h] != -INFINITY;
-      const float pv = used ? __expf(scale * z - S.lse[h]) : 0.f;
-      S.p[h][r] = pv;
-      S.dz[h][r] = pv * (dp - S.dh[h]);
-    }
-    __syncthreads();
-    // dQ += dZ . rows
-#pragma unroll 1
-    for (int r = 0; r < kRT; ++r) {
-      const float g = S.dz[hq][r];
-      const float* src = &S.rows[r][dq0];
+
+    // ---- product 1: z and dO.v of heads 4hb.., rows 4rb.., dim chunks ks, ks+KS, ...
+    {
+      float z[4][4], dp[4][4];
 #pragma unroll
-      for (int j = 0; j < QPER; ++j) dq[j] = fmaf(g, src[j], dq[j]);
-    }
-    // this row's dKV contribution over the chunk's heads, added to the cache gradient
-    const int64_t row = S.row_of[rk];
-    if (row >= 0) {
-      float acc[KPER];
+      for (int a = 0; a < 4; ++a)
 #pragma unroll
-      for (int j = 0; j < KPER; ++j) acc[j] = 0.f;
-#pragma unroll 1
-      for (int h = 0; h < HC; ++h) {
-        const float g = scale * S.dz[h][rk];
-        const float pv = S.p[h][rk];
-        const float* qs = &S.q[h][dk0];
-        const float* os = &S.dout[h][dk0];
+        for (int b = 0; b < 4; ++b) { z[a][b] = 0.f; dp[a][b] = 0.f; }
+#pragma unroll 2
+      for (int c = ks; c < DSA_D_QK / 4; c += KS) {
+        const int d = c * 4;
+        float4 qa[4], ra[4];
 #pragma unroll
-        for (int j = 0; j < KPER; ++j) {
-          acc[j] = fmaf(g, qs[j], acc[j]);
-          if (dk0 + j < DSA_D_V) acc[j] = fmaf(pv, os[j], acc[j]);
+        for (int a = 0; a < 4; ++a) qa[a] = *reinterpret_cast<const float4*>(&S.q[hb * 4 + a][d]);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) ra[b] = *reinterpret_cast<const float4*>(&S.rows[rb * 4 + b][d]);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            z[a][b] = fmaf(qa[a].x, ra[b].x, z[a][b]);
+            z[a][b] = fmaf(qa[a].y, ra[b].y, z[a][b]);
+            z[a][b] = fmaf(qa[a].z, ra[b].z, z[a][b]);
+            z[a][b] = fmaf(qa[a].w, ra[b].w, z[a][b]);
+          }
+        if (d < DSA_D_V) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a) {
+            const float4 oa = *reinterpret_cast<const float4*>(&S.dout[hb * 4 + a][d]);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              dp[a][b] = fmaf(oa.x, ra[b].x, dp[a][b]);
+              dp[a][b] = fmaf(oa.y, ra[b].y, dp[a][b]);
+              dp[a][b] = fmaf(oa.z, ra[b].z, dp[a][b]);
+              dp[a][b] = fmaf(oa.w, ra[b].w, dp[a][b]);
+            }
+          }
         }
       }
-      float* dst = p.d_kv + row * DSA_D_QK + dk0;      // dk0 = 36 * lane-of-row: 16-byte aligned
+      // sum the KS slices (lanes tile*KS .. +KS-1 of one warp)
 #pragma unroll
-      for (int j = 0; j < KPER; j += 4)
-        atomicAdd(reinterpret_cast<float4*>(dst + j), make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]));
+      for (int o = KS / 2; o > 0; o >>= 1)
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            z[a][b] += __shfl_xor_sync(0xffffffffu, z[a][b], o);
+            dp[a][b] += __shfl_xor_sync(0xffffffffu, dp[a][b], o);
+          }
+      // p and dZ: slice lane ks < 4 takes row 4rb + ks
+      if (ks < 4) {
+        const int r = rb * 4 + ks;
+        const bool row_used = S.row_of[r] >= 0;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+          const int h = hb * 4 + a;
+          float zz = z[a][0], dd = dp[a][0];
+#pragma unroll
+          for (int b = 1; b < 4; ++b)
+            if (ks == b) { zz = z[a][b]; dd = dp[a][b]; }
+          const bool used = row_used && S.lse[h] != -INFINITY;
+          const float pv = used ? __expf(scale * zz - S.lse[h]) : 0.f;
+          S.p[h][r] = pv;
+          S.dz[h][r] = pv * (dd - S.dh[h]);
+        }
+      }
     }
     __syncthreads();
-  }
-  float* dqo = p.d_q + (static_cast<int64_t>(t) * H + h0 + hq) * DSA_D_QK + dq0;
+
+    // ---- product 2: dQ += dZ . rows (heads warp*HPW.., dims lane*2 + 64j)
+#pragma unroll 2
+    for (int r = 0; r < kRT; ++r) {
+      float g[HPW];
 #pragma unroll
-  for (int j = 0; j < QPER; ++j) dqo[j] = scale * dq[j];
+      for (int a = 0; a < HPW; ++a) g[a] = S.dz[warp * HPW + a][r];
+#pragma unroll
+      for (int j = 0; j < kDPer / 2; ++j) {
+        const float2 v = *reinterpret_cast<const float2*>(&S.rows[r][lane * 2 + 64 * j]);
+#pragma unroll
+        for (int a = 0; a < HPW; ++a) {
+          dq[a][2 * j] = fmaf(g[a], v.x, dq[a][2 * j]);
+          dq[a][2 * j + 1] = fmaf(g[a], v.y, dq[a][2 * j + 1]);
+        }
+      }
+    }
+
+    // ---- product 3: the d_kv contributions of rows 4*warp.. (dims lane*2 + 64j)
+    {
+      float acc[4][kDPer];
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+#pragma unroll
+        for (int j = 0; j < kDPer; ++j) acc[b][j] = 0.f;
+#pragma unroll 1
+      for (int h = 0; h < HC; ++h) {
+        float g[4], pv[4];
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          g[b] = scale * S.dz[h][warp * 4 + b];
+          pv[b] = S.p[h][warp * 4 + b];
+        }
+#pragma unroll
+        for (int j = 0; j < kDPer / 2; ++j) {
+          const float2 qv = *reinterpret_cast<const float2*>(&S.q[h][lane * 2 + 64 * j]);
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            acc[b][2 * j] = fmaf(g[b], qv.x, acc[b][2 * j]);
+            acc[b][2 * j + 1] = fmaf(g[b], qv.y, acc[b][2 * j + 1]);
+          }
+          if (64 * j < DSA_D_V) {                  // dims 64j + lane*2 < 512 for j < 8
+            const float2 ov = *reinterpret_cast<const float2*>(&S.dout[h][lane * 2 + 64 * j]);
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              acc[b][2 * j] = fmaf(pv[b], ov.x, acc[b][2 * j]);
+              acc[b][2 * j + 1] = fmaf(pv[b], ov.y, acc[b][2 * j + 1]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int64_t row = S.row_of[warp * 4 + b];
+        if (row < 0) continue;
+        float* dst = p.d_kv + row * DSA_D_QK + lane * 2;       // 8-byte aligned
+#pragma unroll
+        for (int j = 0; j < kDPer / 2; ++j)
+          atomicAdd(reinterpret_cast<float2*>(dst + 64 * j), make_float2(acc[b][2 * j], acc[b][2 * j + 1]));
+      }
+    }
+    __syncthreads();                               // rows, p, dz and row_of are rewritten by the next tile
+  }
+#pragma unroll
+  for (int a = 0; a < HPW; ++a) {
+    float* dqo = p.d_q + (static_cast<int64_t>(t) * H + h0 + warp * HPW + a) * DSA_D_QK + lane * 2;
+#pragma unroll
+    for (int j = 0; j < kDPer / 2; ++j)
+      *reinterpret_cast<float2*>(dqo + 64 * j) = make_float2(scale * dq[a][2 * j], scale * dq[a][2 * j + 1]);
+  }
 }
 
 template <int HC>
