@@ -18,7 +18,8 @@
 //      1/KS slice of the 576 (512) dims, float4 loads, the KS slices summed by
 //      shuffles; then p and dZ, one row per slice lane.
 //   2. dQ += dZ . rows: each thread HC/8 heads x 18 dims, accumulated in
-//      registers over all tiles (written once, no atomics).
+//      registers over all tiles (written once, no atomics), dim pairs with one
+//      packed fma.rn.f32x2.
 //   3. each row's d_kv contribution summed over the chunk's heads: each thread 4
 //      rows x 18 dims, added to the fp32 gradient cache with float2 atomics (a
 //      row selected by several queries collects all their contributions).
@@ -229,8 +230,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mla_backward_kernel(MlaBwdPara
         const float2 v = *reinterpret_cast<const float2*>(&S.rows[r][lane * 2 + 64 * j]);
 #pragma unroll
         for (int a = 0; a < HPW; ++a) {
-          dq[a][2 * j] = fmaf(g[a], v.x, dq[a][2 * j]);
-          dq[a][2 * j + 1] = fmaf(g[a], v.y, dq[a][2 * j + 1]);
+          const float2 r2 = ffma2(make_float2(g[a], g[a]), v, make_float2(dq[a][2 * j], dq[a][2 * j + 1]));
+          dq[a][2 * j] = r2.x;
+          dq[a][2 * j + 1] = r2.y;
         }
       }
     }
@@ -255,15 +257,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mla_backward_kernel(MlaBwdPara
           const float2 qv = *reinterpret_cast<const float2*>(&S.q[h][lane * 2 + 64 * j]);
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
-            acc[b][2 * j] = fmaf(g[b], qv.x, acc[b][2 * j]);
-            acc[b][2 * j + 1] = fmaf(g[b], qv.y, acc[b][2 * j + 1]);
+            const float2 r2 = ffma2(make_float2(g[b], g[b]), qv, make_float2(acc[b][2 * j], acc[b][2 * j + 1]));
+            acc[b][2 * j] = r2.x;
+            acc[b][2 * j + 1] = r2.y;
           }
           if (64 * j < DSA_D_V) {                  // dims 64j + lane*2 < 512 for j < 8
             const float2 ov = *reinterpret_cast<const float2*>(&S.dout[h][lane * 2 + 64 * j]);
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-              acc[b][2 * j] = fmaf(pv[b], ov.x, acc[b][2 * j]);
-              acc[b][2 * j + 1] = fmaf(pv[b], ov.y, acc[b][2 * j + 1]);
+              const float2 r2 = ffma2(make_float2(pv[b], pv[b]), ov, make_float2(acc[b][2 * j], acc[b][2 * j + 1]));
+              acc[b][2 * j] = r2.x;
+              acc[b][2 * j + 1] = r2.y;
             }
           }
         }
