@@ -15,7 +15,8 @@
 // converted to fp32); a tile without a usable entry is skipped.  Per tile, three
 // register-tiled products:
 //   1. z and dO.v for every (head, row): each thread a 4-head x 4-row tile over a
-//      1/KS slice of the 576 (512) dims, float4 loads, the KS slices summed by
+//      1/KS slice of the 576 (512) dims, float4 loads, even and odd dims summed
+//      in the two lanes of packed fma.rn.f32x2 pairs, the KS slices summed by
 //      shuffles; then p and dZ, one row per slice lane.
 //   2. dQ += dZ . rows: each thread HC/8 heads x 18 dims, accumulated in
 //      registers over all tiles (written once, no atomics), dim pairs with one
@@ -153,11 +154,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mla_backward_kernel(MlaBwdPara
 
     // ---- product 1: z and dO.v of heads 4hb.., rows 4rb.., dim chunks ks, ks+KS, ...
     {
+      // z and dO.v accumulate even and odd dims in the two lanes of a packed pair
+      float2 z2[4][4], dp2[4][4];
       float z[4][4], dp[4][4];
 #pragma unroll
       for (int a = 0; a < 4; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) { z[a][b] = 0.f; dp[a][b] = 0.f; }
+        for (int b = 0; b < 4; ++b) { z2[a][b] = make_float2(0.f, 0.f); dp2[a][b] = make_float2(0.f, 0.f); }
 #pragma unroll 2
       for (int c = ks; c < DSA_D_QK / 4; c += KS) {
         const int d = c * 4;
@@ -170,10 +173,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mla_backward_kernel(MlaBwdPara
         for (int a = 0; a < 4; ++a)
 #pragma unroll
           for (int b = 0; b < 4; ++b) {
-            z[a][b] = fmaf(qa[a].x, ra[b].x, z[a][b]);
-            z[a][b] = fmaf(qa[a].y, ra[b].y, z[a][b]);
-            z[a][b] = fmaf(qa[a].z, ra[b].z, z[a][b]);
-            z[a][b] = fmaf(qa[a].w, ra[b].w, z[a][b]);
+            z2[a][b] = ffma2(make_float2(qa[a].x, qa[a].y), make_float2(ra[b].x, ra[b].y), z2[a][b]);
+            z2[a][b] = ffma2(make_float2(qa[a].z, qa[a].w), make_float2(ra[b].z, ra[b].w), z2[a][b]);
           }
         if (d < DSA_D_V) {
 #pragma unroll
@@ -181,14 +182,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) mla_backward_kernel(MlaBwdPara
             const float4 oa = *reinterpret_cast<const float4*>(&S.dout[hb * 4 + a][d]);
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-              dp[a][b] = fmaf(oa.x, ra[b].x, dp[a][b]);
-              dp[a][b] = fmaf(oa.y, ra[b].y, dp[a][b]);
-              dp[a][b] = fmaf(oa.z, ra[b].z, dp[a][b]);
-              dp[a][b] = fmaf(oa.w, ra[b].w, dp[a][b]);
+              dp2[a][b] = ffma2(make_float2(oa.x, oa.y), make_float2(ra[b].x, ra[b].y), dp2[a][b]);
+              dp2[a][b] = ffma2(make_float2(oa.z, oa.w), make_float2(ra[b].z, ra[b].w), dp2[a][b]);
             }
           }
         }
       }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          z[a][b] = z2[a][b].x + z2[a][b].y;
+          dp[a][b] = dp2[a][b].x + dp2[a][b].y;
+        }
       // sum the KS slices (lanes tile*KS .. +KS-1 of one warp)
 #pragma unroll
       for (int o = KS / 2; o > 0; o >>= 1)
