@@ -174,6 +174,31 @@ def test_topk_rows_shared_by_a_cluster(cuda_device):
         _topk_case(cuda_device, rows, k)
     _topk_case(cuda_device, base[:3], 100)
 
+
+
+def test_topk_cached_rows_with_a_list(cuda_device):
+    """Many rows of 10240..20480 keys (one CTA per row, the row cached in shared
+    memory): rows whose keys at or above the first pass's threshold bin fit the
+    list take the two later passes and the output over that list, in index order
+    (ties at the threshold included); rows whose list would overflow (few distinct
+    values) or exceed a quarter of the row take the passes over the cache."""
+    rng = np.random.default_rng(14)
+    k = 2048
+    rows = []
+    for t in range(320):                                      # > 2 rows per SM: no cluster
+        n = int(rng.integers(10240, 20481))
+        kind = t % 4
+        if kind == 0:
+            r = rng.standard_normal(n)
+        elif kind == 1:
+            r = np.round(rng.standard_normal(n), 2)           # ties at the threshold
+        elif kind == 2:
+            r = rng.integers(-3, 4, size=n)                   # seven values: the list overflows
+        else:
+            r = np.concatenate([rng.standard_normal(n - 3000), np.full(3000, 4.0)])   # top k all tied
+        rows.append(r.astype(np.float32))
+    _topk_case(cuda_device, rows, k)
+
 # ----------------------------------------------------------------------------- sparse MLA
 
 
