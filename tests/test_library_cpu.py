@@ -35,6 +35,24 @@ def test_library_exports_every_declared_function(lib):
         assert hasattr(lib, n), n
 
 
+def test_binding_constants_match_the_header():
+    """The binding's op codes, status codes, device flags and limits are the
+    header's (the binding restates them for Python callers)."""
+    src = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    defs = {n: int(v) for n, v in re.findall(r"^#define (DSA_\w+) (\d+)u?\b", src, flags=re.M)}
+    enum = {n: int(v) for n, v in re.findall(r"^\s*(DSA_(?:OK|ERR_\w+)) = (\d+)", src, flags=re.M)}
+    ops = {"DSA_OP_INDEXER": B.OP_INDEXER, "DSA_OP_TOPK": B.OP_TOPK, "DSA_OP_SPARSE_MLA": B.OP_SPARSE_MLA,
+           "DSA_OP_FORWARD": B.OP_FORWARD, "DSA_OP_PROJECT": B.OP_PROJECT,
+           "DSA_OP_MLA_BACKWARD": B.OP_MLA_BACKWARD, "DSA_OP_FORWARD_HOST": B.OP_FORWARD_HOST}
+    for name, value in ops.items():
+        assert defs[name] == value, name
+    assert {n: v for n, v in defs.items() if n.startswith("DSA_OP_")} == ops
+    assert defs["DSA_DEV_BAD_QUERY"] == B.DEV_BAD_QUERY and defs["DSA_DEV_BAD_INDEX"] == B.DEV_BAD_INDEX
+    assert defs["DSA_DEV_TIMEOUT"] == B.DEV_TIMEOUT
+    assert defs["DSA_NOALLOC_MAX_Q"] == B.NOALLOC_MAX_Q
+    assert {v: n for n, v in enum.items()} == B.STATUS_NAMES and enum["DSA_OK"] == B.DSA_OK
+
+
 def test_version_and_status_strings(lib):
     assert lib.dsa_abi_version() == 2
     for code, name in B.STATUS_NAMES.items():
