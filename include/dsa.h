@@ -14,11 +14,15 @@
  *
  * Conventions for every call
  *   - Pointers marked (device) are CUDA device pointers; everything else is host.
- *   - The caller owns every buffer and the stream.  The library allocates
- *     nothing and keeps no per-call state; it creates TMA descriptors on the host
- *     per call.  All calls are asynchronous on `stream` (a cudaStream_t passed as
- *     void*; NULL = the legacy default stream) and never synchronise, except
- *     dsa_read_device_status.
+ *   - The caller owns every buffer and the stream.  The library allocates no
+ *     device memory (workspaces are the caller's) and keeps no per-call state;
+ *     it creates TMA descriptors on the host per call.  Kept per device across
+ *     calls: cached kernel attributes, one cuBLASLt handle (created by the first
+ *     dsa_project_append) and the fixed array of dsa_indexer_scores_noalloc;
+ *     dsa_forward_host creates CUDA events for its cross-stream ordering and
+ *     destroys them before it returns.  All calls are asynchronous on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream) and
+ *     never synchronise, except dsa_read_device_status.
  *   - Arguments are checked on the host before any launch; on a failed check
  *     nothing is launched or written and the status says why.
  *   - Errors the host cannot see (a query position beyond its sequence, an index
